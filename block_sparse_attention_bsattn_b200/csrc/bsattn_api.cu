@@ -1,0 +1,246 @@
+// Host side of the C ABI declared in include/bsattn.h: argument validation,
+// TMA tensor-map encoding (through the driver entry point, so the library
+// needs no link-time libcuda), kernel attribute set-up and launches.
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "bsattn.h"
+#include "bsattn_internal.h"
+
+namespace bsattn {
+
+// ------------------------------------------------------------------ debug knobs
+static unsigned long long g_wait_limit_ns = 2000000000ull;  // 2 s
+static int g_inject_stall = 0;
+
+// ------------------------------------------------------------------ driver entry
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                         cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor [Z][Y][X] (X contiguous) tiled in boxes of 64 x box_rows x 1
+// with the 128-byte swizzle; out-of-range rows read as zero.
+static bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t X, uint64_t Y,
+                           uint64_t Z, uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {X, Y, Z};
+  cuuint64_t strides[2] = {X * 2, X * Y * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BSATTN_ERR_CUDA;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return BSATTN_ERR_CUDA;
+  return major == 10 ? BSATTN_OK : BSATTN_ERR_UNSUPPORTED;
+}
+
+static bool bad_lambda(float lambda) { return !(lambda >= 0.f && lambda <= 1.f); }
+
+}  // namespace bsattn
+
+using namespace bsattn;
+
+extern "C" {
+
+const char* bsattn_status_string(int status) {
+  switch (status) {
+    case BSATTN_OK: return "BSATTN_OK";
+    case BSATTN_ERR_INVALID_ARG: return "BSATTN_ERR_INVALID_ARG";
+    case BSATTN_ERR_UNSUPPORTED: return "BSATTN_ERR_UNSUPPORTED";
+    case BSATTN_ERR_ALIGNMENT: return "BSATTN_ERR_ALIGNMENT";
+    case BSATTN_ERR_CAPACITY: return "BSATTN_ERR_CAPACITY";
+    case BSATTN_ERR_CUDA: return "BSATTN_ERR_CUDA";
+    case BSATTN_ERR_DEVICE_TIMEOUT: return "BSATTN_ERR_DEVICE_TIMEOUT";
+    default: return "BSATTN_UNKNOWN_STATUS";
+  }
+}
+
+int bsattn_version(void) { return 100; }
+
+int bsattn_debug_set(long long wait_limit_ns, int inject_stall) {
+  if (wait_limit_ns <= 0) return BSATTN_ERR_INVALID_ARG;
+  g_wait_limit_ns = (unsigned long long)wait_limit_ns;
+  g_inject_stall = inject_stall ? 1 : 0;
+  return BSATTN_OK;
+}
+
+int bsattn_build_index(const uint8_t* d_mask, int mask_heads, int nq_blocks, int nk_blocks,
+                       int q_block, int k_block, int causal, int32_t* d_row_ptr,
+                       int32_t* d_col_idx, int64_t col_capacity, int32_t* d_nnz,
+                       int32_t* d_status, cudaStream_t stream) {
+  if (!d_mask || !d_row_ptr || !d_nnz || (!d_col_idx && col_capacity > 0))
+    return BSATTN_ERR_INVALID_ARG;
+  if (mask_heads < 1 || nq_blocks < 1 || nk_blocks < 1 || q_block < 1 || k_block < 1 ||
+      col_capacity < 0)
+    return BSATTN_ERR_INVALID_ARG;
+  if ((int64_t)mask_heads * nq_blocks * nk_blocks > (int64_t)INT32_MAX)
+    return BSATTN_ERR_UNSUPPORTED;
+  if (int rc = check_device()) return rc;
+  IndexArgs a{d_mask, mask_heads, nq_blocks, nk_blocks, q_block, k_block, causal ? 1 : 0,
+              d_row_ptr, d_col_idx, col_capacity, d_nnz, d_status};
+  return launch_build_index(a, stream) == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}
+
+int bsattn_fwd_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int N, int d, int block, float scale, int causal,
+                       float lambda, const int32_t* row_ptr, const int32_t* col_idx,
+                       int mask_heads, uint8_t* tile_status, int32_t* d_status,
+                       cudaStream_t stream) {
+  if (!q || !k || !v || !o) return BSATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0) return BSATTN_ERR_INVALID_ARG;
+  if (bad_lambda(lambda) || !std::isfinite(scale) || !(scale > 0.f)) return BSATTN_ERR_INVALID_ARG;
+  if (row_ptr && (!col_idx || (mask_heads != 1 && mask_heads != Hq))) return BSATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return BSATTN_ERR_UNSUPPORTED;
+  if (block != 64 && block != 128) return BSATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return BSATTN_ERR_ALIGNMENT;
+  const int64_t nq = (N + block - 1) / block;
+  const int64_t items = (int64_t)B * Hq * nq;
+  if (items > INT32_MAX || (int64_t)B * Hq > INT32_MAX / 2) return BSATTN_ERR_UNSUPPORTED;
+  if (int rc = check_device()) return rc;
+
+  CUtensorMap tq, tk, tv;
+  if (!encode_bf16_3d(&tq, q, d, N, (uint64_t)B * Hq, block) ||
+      !encode_bf16_3d(&tk, k, d, N, (uint64_t)B * Hkv, block) ||
+      !encode_bf16_3d(&tv, v, d, N, (uint64_t)B * Hkv, block))
+    return BSATTN_ERR_CUDA;
+
+  if (tile_status &&
+      cudaMemsetAsync(tile_status, 0, (size_t)items * (size_t)nq, stream) != cudaSuccess)
+    return BSATTN_ERR_CUDA;
+
+  PrefillParams p{};
+  p.row_ptr = row_ptr;
+  p.col_idx = col_idx;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.tile_status = tile_status;
+  p.status = d_status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.nq = (int)nq;
+  p.nk = (int)nq;
+  p.mask_heads = mask_heads;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  p.use_skip = lambda > 0.f ? 1 : 0;
+  p.thr_log2 = lambda > 0.f ? (float)std::log2((double)lambda) : -INFINITY;
+  p.debug_stall = g_inject_stall;
+  p.wait_limit_ns = g_wait_limit_ns;
+
+  cudaError_t e;
+  if (d == 128 && block == 128) e = launch_prefill<128, 128>(tq, tk, tv, p, (int)items, stream);
+  else if (d == 64 && block == 128) e = launch_prefill<64, 128>(tq, tk, tv, p, (int)items, stream);
+  else if (d == 128 && block == 64) e = launch_prefill<128, 64>(tq, tk, tv, p, (int)items, stream);
+  else e = launch_prefill<64, 64>(tq, tk, tv, p, (int)items, stream);
+  return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}
+
+size_t bsattn_decode_workspace_size(int B, int Hq, int d, int num_splits) {
+  if (B < 1 || Hq < 1 || d < 1 || num_splits < 1) return 0;
+  const size_t rows = (size_t)B * Hq * num_splits;
+  return rows * (size_t)d * 4 + rows * 4 * 2;
+}
+
+int bsattn_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int Hq, int Hkv, int L, int d, int block, float scale, int causal,
+                      float lambda, int num_splits, void* workspace, size_t workspace_bytes,
+                      uint8_t* tile_status, int32_t* d_status, cudaStream_t stream) {
+  (void)causal;
+  if (!q || !k || !v || !o || !workspace) return BSATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0 || num_splits < 1)
+    return BSATTN_ERR_INVALID_ARG;
+  if (bad_lambda(lambda) || !std::isfinite(scale) || !(scale > 0.f)) return BSATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return BSATTN_ERR_UNSUPPORTED;
+  if (block != 64 && block != 128) return BSATTN_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return BSATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(workspace))
+    return BSATTN_ERR_ALIGNMENT;
+  if (workspace_bytes < bsattn_decode_workspace_size(B, Hq, d, num_splits))
+    return BSATTN_ERR_CAPACITY;
+  const int T = (L + block - 1) / block;
+  const int64_t grid = (int64_t)B * Hkv * num_splits;
+  if (grid > INT32_MAX || (int64_t)B * Hq > INT32_MAX) return BSATTN_ERR_UNSUPPORTED;
+  if (int rc = check_device()) return rc;
+
+  CUtensorMap tk, tv;
+  if (!encode_bf16_3d(&tk, k, d, L, (uint64_t)B * Hkv, block) ||
+      !encode_bf16_3d(&tv, v, d, L, (uint64_t)B * Hkv, block))
+    return BSATTN_ERR_CUDA;
+  if (tile_status &&
+      cudaMemsetAsync(tile_status, 0, (size_t)B * Hkv * (size_t)T, stream) != cudaSuccess)
+    return BSATTN_ERR_CUDA;
+
+  const size_t rows = (size_t)B * Hq * num_splits;
+  DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_m = p.ws_o + rows * d;
+  p.ws_l = p.ws_m + rows;
+  p.tile_status = tile_status;
+  p.status = d_status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.L = L;
+  p.T = T;
+  p.splits = num_splits;
+  p.chunk = (T + num_splits - 1) / num_splits;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  p.use_skip = lambda > 0.f ? 1 : 0;
+  p.thr_log2 = lambda > 0.f ? (float)std::log2((double)lambda) : -INFINITY;
+  p.wait_limit_ns = g_wait_limit_ns;
+
+  cudaError_t e = cudaErrorInvalidValue;
+#define BSATTN_DEC(DD, BB, GG)                                               \
+  if (d == DD && block == BB && G == GG)                                     \
+    e = launch_decode_split<DD, BB, GG>(tk, tv, p, (int)grid, stream);
+  BSATTN_DEC(128, 128, 1) BSATTN_DEC(128, 128, 2) BSATTN_DEC(128, 128, 4) BSATTN_DEC(128, 128, 8)
+  BSATTN_DEC(64, 128, 1) BSATTN_DEC(64, 128, 2) BSATTN_DEC(64, 128, 4) BSATTN_DEC(64, 128, 8)
+  BSATTN_DEC(128, 64, 1) BSATTN_DEC(128, 64, 2) BSATTN_DEC(128, 64, 4) BSATTN_DEC(128, 64, 8)
+  BSATTN_DEC(64, 64, 1) BSATTN_DEC(64, 64, 2) BSATTN_DEC(64, 64, 4) BSATTN_DEC(64, 64, 8)
+#undef BSATTN_DEC
+  if (e != cudaSuccess) return BSATTN_ERR_CUDA;
+
+  CombineParams c{p.ws_o, p.ws_m, p.ws_l, static_cast<__nv_bfloat16*>(o), lse, num_splits, d};
+  e = launch_decode_combine(c, B * Hq, d, stream);
+  return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,433 @@
+// Block-sparse attention prefill for sm_100a: tcgen05 tensor-core MMAs with
+// TMEM accumulators, TMA-staged tiles, warp-specialised roles, and the BLASST
+// skip test inside the online softmax.
+//
+// What it computes ("BLASST: Dynamic Blocked Attention Sparsity via Softmax
+// Thresholding", Algorithm 1 and section 4.1; "块稀疏Attention实战" section
+// 3.3): for each query tile, the key tiles of its visit list are processed in
+// ascending order; every visited tile gets S = Q K^T (BMM1), its row max, and
+// the skip test against the running max; a kept tile then gets P = exp(S - m)
+// (CUDA cores), the row sums, and O += P V (BMM2).  A skipped tile costs one
+// BMM1 and a row max.
+//
+// One CTA = one (batch, head, query tile) work item; 6 warps:
+//   warp 0      TMA producer: Q once, then K_j and V_j of every visited tile
+//               into 2-stage rings (V is loaded for every visited tile, as the
+//               BLASST prefill kernel does -- the load is not on the critical
+//               path of a compute-bound kernel);
+//   warp 1      TMEM owner and MMA issuer (one elected lane): BMM1 of tile
+//               t + 1 is issued before waiting for the softmax of tile t, so
+//               the tensor core works while the softmax warps do;
+//   warps 2..5  softmax: one thread per query row (TMEM lane), skip vote
+//               (__all_sync per warp, then one shared-memory flag and one
+//               mbarrier arrival per warp to agree across the four warps),
+//               P = exp2 written back to
+//               TMEM as bf16 over the tile's S columns, lazy rescale of O, and
+//               the epilogue.
+// TMEM columns: S double buffer at [0,128) and [128,256), O at [256, 256+d).
+// BMM1: A = Q (smem, K-major, 128B swizzle), B = K tile (smem, K-major).
+// BMM2: A = P (TMEM), B = V tile (smem, MN-major, 128B swizzle).
+// The query tile always occupies 128 MMA rows; with 64-token tiles rows
+// 64..127 carry no data and their outputs are never read.
+#include <cmath>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "bsattn_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace bsattn {
+
+template <int D, int BLK>
+struct PrefillCfg {
+  static constexpr int KST = 2;                    // K ring stages
+  static constexpr int VST = 2;                    // V ring stages
+  static constexpr int HALVES = D / 64;            // 64-column (128-byte) swizzle boxes
+  static constexpr int Q_HALF = 128 * 128;         // bytes per Q box region (128 rows)
+  static constexpr int T_HALF = BLK * 128;         // bytes per K/V box region
+  static constexpr int Q_BYTES = HALVES * Q_HALF;
+  static constexpr int T_BYTES = HALVES * T_HALF;
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + Q_BYTES;
+  static constexpr int V_OFF = K_OFF + KST * T_BYTES;
+  static constexpr int BAR_OFF = V_OFF + VST * T_BYTES;
+  // + alignment slack; at least 116 KB so that one CTA (which holds all 512
+  // TMEM columns) is resident per SM
+  static constexpr int SMEM_USED = BAR_OFF + 256 + 1024;
+  static constexpr int SMEM = SMEM_USED > 118784 ? SMEM_USED : 118784;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t S_COL = 0;             // S[b] at b * 128
+  static constexpr uint32_t O_COL = 256;
+  static constexpr int THREADS = 192;
+  static constexpr float TAU = 8.0f;               // lazy-rescale slack (base-2 units)
+};
+
+struct PrefillBarriers {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2];
+  uint64_t v_full[2], v_empty[2];
+  uint64_t s_full[2];
+  uint64_t p_ready[2];
+  uint64_t o_done;
+  uint64_t drain;
+  uint64_t vote_bar[2];
+  uint32_t tmem_base;
+  int abort;
+  int skip_flag[2];
+  int vote[2][4];
+};
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(192, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+  using C = PrefillCfg<D, BLK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* q_smem = smem + C::Q_OFF;
+  uint8_t* k_smem = smem + C::K_OFF;
+  uint8_t* v_smem = smem + C::V_OFF;
+  PrefillBarriers* bars = reinterpret_cast<PrefillBarriers*>(smem + C::BAR_OFF);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  // ---- work item (longest-first for causal: query tiles in descending order)
+  const int BH = p.B * p.Hq;
+  int i, bh;
+  if (p.causal) {
+    i = p.nq - 1 - (int)(blockIdx.x / BH);
+    bh = (int)(blockIdx.x % BH);
+  } else {
+    bh = (int)(blockIdx.x / p.nq);
+    i = (int)(blockIdx.x % p.nq);
+  }
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int kvh = h / (p.Hq / p.Hkv);
+
+  // ---- visit list
+  const int32_t* cols = nullptr;
+  int n;
+  if (p.row_ptr) {
+    const int mh = p.mask_heads == 1 ? 0 : h;
+    const int32_t s0 = p.row_ptr[(int64_t)mh * (p.nq + 1) + i];
+    const int32_t s1 = p.row_ptr[(int64_t)mh * (p.nq + 1) + i + 1];
+    cols = p.col_idx + s0;
+    n = s1 - s0;
+    if (p.causal)
+      while (n > 0 && cols[n - 1] > i) --n;
+  } else {
+    n = p.causal ? i + 1 : p.nk;
+  }
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->p_ready[s], 4);
+    }
+    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->vote_bar[0], 4);
+    mbar_init(&bars->vote_bar[1], 4);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const uint64_t lim = p.wait_limit_ns;
+
+  if (warp == 0) {
+    // ======================================================== TMA producer
+    if (lane == 0 && n > 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      if (!p.debug_stall) {
+        mbar_arrive_expect_tx(&bars->q_full, C::HALVES * BLK * 128);
+        for (int hf = 0; hf < C::HALVES; ++hf)
+          tma_load_3d(q_smem + hf * C::Q_HALF, &tmQ, &bars->q_full, hf * 64, i * BLK,
+                      b * p.Hq + h);
+      }
+      int issued_k = 0, issued_v = 0;
+      for (int t = 0; t < n; ++t) {
+        const int j = cols ? cols[t] : t;
+        const int ks = t % C::KST;
+        if (!mbar_wait(&bars->k_empty[ks], ((t / C::KST) & 1) ^ 1, abort, lim)) break;
+        mbar_arrive_expect_tx(&bars->k_full[ks], C::T_BYTES);
+        for (int hf = 0; hf < C::HALVES; ++hf)
+          tma_load_3d(k_smem + ks * C::T_BYTES + hf * C::T_HALF, &tmK, &bars->k_full[ks],
+                      hf * 64, j * BLK, b * p.Hkv + kvh);
+        ++issued_k;
+        const int vs = t % C::VST;
+        if (!mbar_wait(&bars->v_empty[vs], ((t / C::VST) & 1) ^ 1, abort, lim)) break;
+        mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
+        for (int hf = 0; hf < C::HALVES; ++hf)
+          tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
+                      hf * 64, j * BLK, b * p.Hkv + kvh);
+        ++issued_v;
+      }
+      if (*abort) {
+        // let every copy this thread started land before the CTA can exit
+        for (int t = (issued_k > C::KST ? issued_k - C::KST : 0); t < issued_k; ++t)
+          mbar_wait_drain(&bars->k_full[t % C::KST], (t / C::KST) & 1, lim);
+        for (int t = (issued_v > C::VST ? issued_v - C::VST : 0); t < issued_v; ++t)
+          mbar_wait_drain(&bars->v_full[t % C::VST], (t / C::VST) & 1, lim);
+        if (!p.debug_stall)
+          mbar_wait_drain(&bars->q_full, 0, lim);
+      }
+    }
+  } else if (warp == 1) {
+    // ======================================================== MMA issuer
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t IDESC1 = idesc_bf16_f32(128, BLK, 0, 0);
+      constexpr uint32_t IDESC2 = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_addr = smem_u32(q_smem);
+      const uint32_t k_addr = smem_u32(k_smem);
+      const uint32_t v_addr = smem_u32(v_smem);
+      bool ok = mbar_wait(&bars->q_full, 0, abort, lim);
+      tc_fence_after();
+      auto issue_bmm1 = [&](int t) -> bool {
+        const int ks = t % C::KST;
+        if (!mbar_wait(&bars->k_full[ks], (t / C::KST) & 1, abort, lim)) return false;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + C::S_COL + (uint32_t)(t & 1) * 128u;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t a = q_addr + (kk / 4) * C::Q_HALF + (kk % 4) * 32;
+          const uint32_t bb = k_addr + ks * C::T_BYTES + (kk / 4) * C::T_HALF + (kk % 4) * 32;
+          mma_ss(d_tmem, smem_desc(a, 16, 1024, 2), smem_desc(bb, 16, 1024, 2), IDESC1,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->s_full[t & 1]);
+        mma_commit(&bars->k_empty[ks]);
+        return true;
+      };
+      if (ok) ok = issue_bmm1(0);
+      int kept = 0;
+      for (int t = 0; ok && t < n; ++t) {
+        if (t + 1 < n && !issue_bmm1(t + 1)) break;
+        const int sb = t & 1;
+        if (!mbar_wait(&bars->p_ready[sb], (t >> 1) & 1, abort, lim)) break;
+        tc_fence_after();
+        const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[sb]);
+        const int vs = t % C::VST;
+        if (!mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) break;
+        tc_fence_after();
+        if (!skip) {
+          const uint32_t p_tmem = tmem + C::S_COL + (uint32_t)sb * 128u;
+#pragma unroll
+          for (int kk = 0; kk < BLK / 16; ++kk) {
+            const uint32_t bb = v_addr + vs * C::T_BYTES + kk * (16 * 128);
+            mma_ts(tmem + C::O_COL, p_tmem + kk * 8, smem_desc(bb, C::T_HALF, 1024, 2), IDESC2,
+                   (kept > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bars->o_done);
+          mma_commit(&bars->v_empty[vs]);
+          ++kept;
+        } else {
+          mbar_arrive(&bars->v_empty[vs]);
+        }
+      }
+      // all tcgen05 work issued by this thread must finish before TMEM is freed
+      mma_commit(&bars->drain);
+      mbar_wait_drain(&bars->drain, 0, lim);
+    }
+  } else {
+    // ======================================================== softmax warps
+    const int quarter = warp % 4;           // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;    // query row inside the tile
+    const int r0 = i * BLK;
+    const bool in_tile = row < BLK;
+    const bool valid = in_tile && (r0 + row < p.N);
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int sw = warp - 2;                // 0..3
+    float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
+    int kept = 0;
+    bool ok = true;
+    for (int t = 0; t < n; ++t) {
+      const int j = cols ? cols[t] : t;
+      const int sb = t & 1;
+      if (!mbar_wait(&bars->s_full[sb], (t >> 1) & 1, abort, lim)) { ok = false; break; }
+      tc_fence_after();
+      float s[BLK];
+      if (in_tile) {
+#pragma unroll
+        for (int c0 = 0; c0 < BLK; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(lane_addr + C::S_COL + sb * 128 + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) s[c0 + c] = __uint_as_float(r[c]);
+        }
+        // element masks: keys past the end, and keys after the query (causal)
+        const int k0 = j * BLK;
+        if (k0 + BLK > p.N || (p.causal && j == i)) {
+          const int qpos = r0 + row;
+#pragma unroll
+          for (int c = 0; c < BLK; ++c) {
+            const int key = k0 + c;
+            if (key >= p.N || (p.causal && key > qpos)) s[c] = -INFINITY;
+          }
+        }
+      }
+      float mx = -INFINITY;
+      if (in_tile) {
+#pragma unroll
+        for (int c = 0; c < BLK; ++c) mx = fmaxf(mx, s[c]);
+      }
+      const float mt = mx * p.scale_log2;  // tile row max, base-2 units
+      int skip = 0;
+      if (p.use_skip) {
+        // skip only if every valid row is below the running max + log2(lambda)
+        const bool pass = !valid || (mt - m_run < p.thr_log2);
+        const bool wpass = __all_sync(0xffffffffu, pass);
+        if (lane == 0) {
+          bars->vote[t & 1][sw] = wpass ? 1 : 0;
+          mbar_arrive(&bars->vote_bar[t & 1]);
+        }
+        __syncwarp();
+        if (!mbar_wait(&bars->vote_bar[t & 1], (t >> 1) & 1, abort, lim)) { ok = false; break; }
+        volatile int* vv = bars->vote[t & 1];
+        skip = vv[0] & vv[1] & vv[2] & vv[3];
+      }
+      m_run = fmaxf(m_run, mt);
+      if (sw == 0 && lane == 0 && p.tile_status && (unsigned)j < (unsigned)p.nk)
+        p.tile_status[(((int64_t)b * p.Hq + h) * p.nq + i) * p.nk + j] = skip ? 1 : 2;
+      if (!skip) {
+        if (kept > 0) {
+          // the previous BMM2 must be complete before P overwrites this S
+          // buffer's neighbour state and before O may be rescaled
+          if (!mbar_wait(&bars->o_done, (kept - 1) & 1, abort, lim)) { ok = false; break; }
+          tc_fence_after();
+        }
+        float m_new = m_ref;
+        if (kept == 0) {
+          m_new = m_run;
+        } else if (m_run > m_ref + C::TAU) {
+          m_new = m_run;
+          const float alpha = fast_exp2(m_ref - m_new);
+          l *= alpha;
+          if (in_tile) {
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t r[32];
+              tmem_ld32(lane_addr + C::O_COL + c0, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+              tmem_st32(lane_addr + C::O_COL + c0, r);
+            }
+            tmem_wait_st();
+          }
+        }
+        m_ref = m_new;
+        const float shift = (m_ref == -INFINITY) ? 0.f : m_ref;
+        if (in_tile) {
+          float rs = 0.f;
+#pragma unroll
+          for (int c0 = 0; c0 < BLK; c0 += 32) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const float p0 = fast_exp2(fmaf(s[c0 + c], p.scale_log2, -shift));
+              const float p1 = fast_exp2(fmaf(s[c0 + c + 1], p.scale_log2, -shift));
+              rs += p0 + p1;
+              pk[c / 2] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(lane_addr + C::S_COL + sb * 128 + c0 / 2, pk);
+          }
+          tmem_wait_st();
+          l += rs;
+        }
+        ++kept;
+      }
+      if (sw == 0 && lane == 0) bars->skip_flag[sb] = skip;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_ready[sb]);
+    }
+
+    // ---- epilogue: O / l -> bf16, LSE
+    if (ok && kept > 0) {
+      if (!mbar_wait(&bars->o_done, (kept - 1) & 1, abort, lim)) ok = false;
+      tc_fence_after();
+    }
+    if (ok && valid) {
+      const int64_t orow = ((int64_t)b * p.Hq + h) * p.N + r0 + row;
+      __nv_bfloat16* dst = p.o + orow * D;
+      const bool have = kept > 0 && l > 0.f;
+      const float inv_l = have ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
+        if (kept > 0) {
+          tmem_ld32(lane_addr + C::O_COL + c0, r);
+          tmem_wait_ld();
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float a0 = have ? __uint_as_float(r[c]) * inv_l : 0.f;
+          const float a1 = have ? __uint_as_float(r[c + 1]) * inv_l : 0.f;
+          w[c / 2] = pack_bf16x2(a0, a1);
+        }
+        uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+      }
+      if (p.lse) p.lse[orow] = have ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && bars->abort) report_status(p.status, kDevTimeout);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D, int BLK>
+cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const PrefillParams& p, int grid, cudaStream_t stream) {
+  using C = PrefillCfg<D, BLK>;
+  static_assert(C::SMEM <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, BLK>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  prefill_kernel<D, BLK><<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_prefill<128, 128>(const CUtensorMap&, const CUtensorMap&,
+                                              const CUtensorMap&, const PrefillParams&, int,
+                                              cudaStream_t);
+template cudaError_t launch_prefill<64, 128>(const CUtensorMap&, const CUtensorMap&,
+                                             const CUtensorMap&, const PrefillParams&, int,
+                                             cudaStream_t);
+template cudaError_t launch_prefill<128, 64>(const CUtensorMap&, const CUtensorMap&,
+                                             const CUtensorMap&, const PrefillParams&, int,
+                                             cudaStream_t);
+template cudaError_t launch_prefill<64, 64>(const CUtensorMap&, const CUtensorMap&,
+                                            const CUtensorMap&, const PrefillParams&, int,
+                                            cudaStream_t);
+
+}  // namespace bsattn

@@ -1,0 +1,176 @@
+"""ctypes binding of the C ABI in ``include/bsattn.h`` -- argument marshalling only.
+
+Every function here takes torch tensors on the current CUDA device, checks
+shapes/dtypes, allocates outputs the caller did not pass, and calls the entry
+point of the same name in ``lib/libbsattn.so`` on the current torch stream.
+All arithmetic happens in the library's kernels; there is no fallback: if the
+library is missing this module fails to import.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libbsattn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -m block_sparse_attention_bsattn_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+_lib.bsattn_status_string.argtypes = [_I]
+_lib.bsattn_status_string.restype = ctypes.c_char_p
+_lib.bsattn_version.restype = _I
+_lib.bsattn_debug_set.argtypes = [ctypes.c_longlong, _I]
+_lib.bsattn_debug_set.restype = _I
+_lib.bsattn_build_index.argtypes = [_P, _I, _I, _I, _I, _I, _I, _P, _P, _I64, _P, _P, _P]
+_lib.bsattn_build_index.restype = _I
+_lib.bsattn_fwd_prefill.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F,
+                                    _P, _P, _I, _P, _P, _P]
+_lib.bsattn_fwd_prefill.restype = _I
+_lib.bsattn_decode_workspace_size.argtypes = [_I, _I, _I, _I]
+_lib.bsattn_decode_workspace_size.restype = _SZ
+_lib.bsattn_fwd_decode.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F, _I,
+                                   _P, _SZ, _P, _P, _P]
+_lib.bsattn_fwd_decode.restype = _I
+
+EXPORTED = ("bsattn_status_string", "bsattn_version", "bsattn_debug_set", "bsattn_build_index",
+            "bsattn_fwd_prefill", "bsattn_decode_workspace_size", "bsattn_fwd_decode")
+
+
+class BsattnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {bsattn_status_string(code)} ({code})")
+
+
+def bsattn_status_string(code: int) -> str:
+    return _lib.bsattn_status_string(int(code)).decode()
+
+
+def bsattn_version() -> int:
+    return int(_lib.bsattn_version())
+
+
+def bsattn_debug_set(wait_limit_ns: int = 2_000_000_000, inject_stall: bool = False) -> None:
+    """Test hook: per-wait time limit of the pipelined kernels and a switch
+    that makes the prefill producer never issue its first load."""
+    rc = _lib.bsattn_debug_set(int(wait_limit_ns), int(bool(inject_stall)))
+    if rc:
+        raise BsattnError(rc, "bsattn_debug_set")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(t: torch.Tensor, name: str, dtype, dims: int):
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or t.dim() != dims or not t.is_cuda \
+            or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor with {dims} dims")
+
+
+def bsattn_build_index(mask: torch.Tensor, q_block: int, k_block: int, causal: bool = False,
+                       capacity: Optional[int] = None, status: Optional[torch.Tensor] = None,
+                       stream=None):
+    """mask uint8 [mask_heads, nq, nk] -> (row_ptr int32 [mask_heads*(nq+1)],
+    col_idx int32 [capacity], nnz int32 [mask_heads]); col_idx is sized to
+    `capacity` (default: every block)."""
+    if mask.dim() == 2:
+        mask = mask[None]
+    _check(mask, "mask", torch.uint8, 3)
+    Hm, nq, nk = mask.shape
+    cap = Hm * nq * nk if capacity is None else int(capacity)
+    dev = mask.device
+    row_ptr = torch.empty(Hm * (nq + 1), dtype=torch.int32, device=dev)
+    col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
+    nnz = torch.empty(Hm, dtype=torch.int32, device=dev)
+    rc = _lib.bsattn_build_index(_ptr(mask), Hm, nq, nk, int(q_block), int(k_block), int(causal),
+                                 _ptr(row_ptr), _ptr(col_idx), cap, _ptr(nnz), _ptr(status),
+                                 _stream(stream))
+    if rc:
+        raise BsattnError(rc, "bsattn_build_index")
+    return row_ptr, col_idx, nnz
+
+
+def bsattn_fwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int,
+                       scale: Optional[float] = None, causal: bool = False, lam: float = 0.0,
+                       row_ptr: Optional[torch.Tensor] = None,
+                       col_idx: Optional[torch.Tensor] = None, mask_heads: int = 1,
+                       o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                       want_lse: bool = True, tile_status: Optional[torch.Tensor] = None,
+                       status: Optional[torch.Tensor] = None, stream=None):
+    """q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 -> (o [B,Hq,N,d] bf16, lse [B,Hq,N] fp32 or None)."""
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError("k/v must be [B, Hkv, N, d] matching q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
+    rc = _lib.bsattn_fwd_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
+                                 int(block), float(scale), int(causal), float(lam), _ptr(row_ptr),
+                                 _ptr(col_idx), int(mask_heads), _ptr(tile_status), _ptr(status),
+                                 _stream(stream))
+    if rc:
+        raise BsattnError(rc, "bsattn_fwd_prefill")
+    return o, lse
+
+
+def bsattn_decode_workspace_size(B: int, Hq: int, d: int, num_splits: int) -> int:
+    return int(_lib.bsattn_decode_workspace_size(B, Hq, d, num_splits))
+
+
+def bsattn_fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int,
+                      num_splits: int, scale: Optional[float] = None, lam: float = 0.0,
+                      o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                      want_lse: bool = True, workspace: Optional[torch.Tensor] = None,
+                      tile_status: Optional[torch.Tensor] = None,
+                      status: Optional[torch.Tensor] = None, stream=None):
+    """q [B,Hq,d], k/v [B,Hkv,L,d] bf16 -> (o [B,Hq,d] bf16, lse [B,Hq] fp32 or None)."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k, "k", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    B, Hq, d = q.shape
+    Hkv, L = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, L, d) or v.shape != k.shape:
+        raise ValueError("k/v must be [B, Hkv, L, d] matching q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    need = bsattn_decode_workspace_size(B, Hq, d, num_splits)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    rc = _lib.bsattn_fwd_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, L, d,
+                                int(block), float(scale), 0, float(lam), int(num_splits),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _ptr(tile_status), _ptr(status), _stream(stream))
+    if rc:
+        raise BsattnError(rc, "bsattn_fwd_decode")
+    return o, lse

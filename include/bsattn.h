@@ -1,0 +1,163 @@
+/*
+ * bsattn.h -- C ABI of the B200 (sm_100a) block-sparse attention library.
+ *
+ * The library computes the attention forward pass
+ *     O = softmax(scale * Q K^T + M) V
+ * where M removes (a) the key blocks that a static 0/1 block mask zeroes out
+ * ("块稀疏Attention实战", section 2.1: a zero block takes no part in QK,
+ * softmax or PV; section 3.3: the tiling loop checks each block before loading
+ * K) and (b) the key tiles that the BLASST rule skips ("BLASST: Dynamic
+ * Blocked Attention Sparsity via Softmax Thresholding", section 3.1 and
+ * Algorithm 1): inside the online softmax, key tiles of a query tile are
+ * visited in ascending order, and a tile is skipped -- no exp, no row sum, no
+ * P*V -- when, for every valid row of the query tile, the tile's row max is
+ * below the running row max (taken over all earlier visited tiles, skipped or
+ * not) plus ln(lambda).  The output is the exact softmax over the keys of the
+ * executed tiles.
+ *
+ * Conventions shared by every entry point:
+ *  - Tensors are dense and row-major.  Q is [B, Hq, N, d], K and V are
+ *    [B, Hkv, N, d], O is [B, Hq, N, d], all bf16; LSE is [B, Hq, N] fp32
+ *    (natural log of the softmax denominator of the scaled scores).
+ *  - GQA ("Attention 的七十二变", section 5.3-5.4): query head h reads KV head
+ *    h / (Hq / Hkv).
+ *  - All pointers are device pointers unless stated otherwise.  The caller
+ *    allocates and owns every buffer; the library allocates no device memory
+ *    and keeps no state between calls besides a per-device cache of kernel
+ *    attributes.
+ *  - Every call is asynchronous on `stream`.  The return value reports only
+ *    host-side validation and launch errors; nothing is launched when it is
+ *    not BSATTN_OK.  Errors found on the device (a pipeline wait that ran out
+ *    of time, an index capacity overflow) are written to the optional device
+ *    word `d_status`, which the caller sets to 0 beforehand; the library only
+ *    ever writes a nonzero code there.
+ *  - lambda = 0 turns the dynamic skip off; lambda must lie in [0, 1].
+ */
+#ifndef BSATTN_H_
+#define BSATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSATTN_OK = 0,
+  BSATTN_ERR_INVALID_ARG = -1,   /* null pointer, bad size or lambda outside [0, 1] */
+  BSATTN_ERR_UNSUPPORTED = -2,   /* d or block not in {64, 128}, or no sm_100 device */
+  BSATTN_ERR_ALIGNMENT = -3,     /* a tensor pointer is not 16-byte aligned */
+  BSATTN_ERR_CAPACITY = -4,      /* index or workspace too small */
+  BSATTN_ERR_CUDA = -5,          /* a CUDA runtime/driver call failed */
+  BSATTN_ERR_DEVICE_TIMEOUT = -6 /* (device status only) a pipeline wait timed out */
+} bsattn_status;
+
+/* Human-readable name of a status code; never NULL. */
+const char *bsattn_status_string(int status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int bsattn_version(void);
+
+/*
+ * bsattn_debug_set -- test hook, process-wide.  wait_limit_ns bounds every
+ * pipeline wait inside the kernels (default 2 s); when one runs out the kernel
+ * stops, drains its own copies, frees its tensor memory and reports
+ * BSATTN_ERR_DEVICE_TIMEOUT through d_status.  inject_stall != 0 makes the
+ * prefill producer skip its first load so that the limit is reached on
+ * purpose.  Returns BSATTN_ERR_INVALID_ARG for wait_limit_ns <= 0.
+ */
+int bsattn_debug_set(long long wait_limit_ns, int inject_stall);
+
+/*
+ * bsattn_build_index -- block mask -> per-query-block CSR lists.
+ *
+ * Follows "块稀疏Attention实战" section 2.3 (keep the mask as an index of its
+ * non-zero blocks) in the form the prefill kernel walks: for mask head h and
+ * query block i, the key blocks j with mask[h][i][j] != 0, ascending; when
+ * `causal` is set, only those with j * k_block <= (i + 1) * q_block - 1.
+ *
+ *   d_mask      uint8 [mask_heads][nq_blocks][nk_blocks], nonzero = keep
+ *   d_row_ptr   int32 [mask_heads][nq_blocks + 1]: absolute offsets into
+ *               d_col_idx (head h's rows follow head h-1's)
+ *   d_col_idx   int32 [col_capacity]
+ *   d_nnz       int32 [mask_heads]: kept blocks per mask head (always written)
+ *
+ * When the kept blocks exceed col_capacity, no col_idx entry past the
+ * capacity is written and *d_status (if given) receives BSATTN_ERR_CAPACITY;
+ * row_ptr and nnz still describe the full index.  A capacity of
+ * mask_heads * nq_blocks * nk_blocks can never overflow.
+ */
+int bsattn_build_index(const uint8_t *d_mask, int mask_heads, int nq_blocks, int nk_blocks,
+                       int q_block, int k_block, int causal, int32_t *d_row_ptr,
+                       int32_t *d_col_idx, int64_t col_capacity, int32_t *d_nnz,
+                       int32_t *d_status, cudaStream_t stream);
+
+/*
+ * bsattn_fwd_prefill -- block-sparse attention over a whole sequence.
+ *
+ * Query tiles and key tiles are both `block` tokens (64 or 128); d is 64 or
+ * 128.  Query tile i of head h visits, in ascending order, the key tiles of
+ * CSR row i of mask head (mask_heads == 1 ? 0 : h) -- or every key tile when
+ * row_ptr is NULL -- restricted to j <= i when causal.  Inside a visited tile
+ * keys past N and (causal) keys after the query are masked element by
+ * element.  With lambda > 0 each visited tile is tested by the BLASST rule
+ * (all valid rows must pass).  Query rows past N are neither written nor part
+ * of the vote.
+ *
+ *   q, k, v, o      bf16, 16-byte aligned, shapes as in the conventions above
+ *   lse             fp32 [B][Hq][N] or NULL
+ *   scale           softmax scale applied to Q K^T (e.g. 1/sqrt(d))
+ *   row_ptr/col_idx CSR from bsattn_build_index (q_block = k_block = block),
+ *                   or row_ptr = NULL for every tile
+ *   tile_status     uint8 [B][Hq][nq][nk] or NULL; the call first clears it,
+ *                   then writes 1 for each visited-and-skipped tile and 2 for
+ *                   each executed tile (0 = not visited)
+ *   d_status        int32 device word or NULL (see conventions)
+ *
+ * A query row with no executed key gets O = 0 and LSE = -inf.
+ */
+int bsattn_fwd_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
+                       int B, int Hq, int Hkv, int N, int d, int block, float scale, int causal,
+                       float lambda, const int32_t *row_ptr, const int32_t *col_idx,
+                       int mask_heads, uint8_t *tile_status, int32_t *d_status,
+                       cudaStream_t stream);
+
+/*
+ * bsattn_decode_workspace_size -- bytes of scratch bsattn_fwd_decode needs:
+ * per (batch, query head, split) d fp32 partial outputs plus the split's
+ * running max and row sum.
+ */
+size_t bsattn_decode_workspace_size(int B, int Hq, int d, int num_splits);
+
+/*
+ * bsattn_fwd_decode -- one query token per sequence against a KV cache,
+ * split-KV with a combine step.
+ *
+ * The query tile of (batch b, KV head g) is the Hq/Hkv query heads that share
+ * the KV head (their V tile is shared, so it is skipped only when all of them
+ * pass).  The ceil(L / block) key tiles are cut into num_splits contiguous
+ * chunks of ceil(T / num_splits) tiles; each chunk runs the BLASST visit and
+ * test with its own running max starting at -inf (the pages do not define
+ * split-KV; this is the reading this library implements), streaming each K
+ * tile and loading a V tile only when the tile is executed.  A combine kernel
+ * then merges the chunks exactly (log-sum-exp).
+ *
+ *   q           bf16 [B][Hq][d];  k, v bf16 [B][Hkv][L][d]
+ *   o           bf16 [B][Hq][d];  lse fp32 [B][Hq] or NULL
+ *   causal      accepted and ignored: the single query is the last position
+ *   workspace   device scratch of at least bsattn_decode_workspace_size(...)
+ *               bytes, 16-byte aligned, owned by the caller
+ *   tile_status uint8 [B][Hkv][T] or NULL (cleared, then 1 skipped / 2 executed)
+ */
+int bsattn_fwd_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                      int Hq, int Hkv, int L, int d, int block, float scale, int causal,
+                      float lambda, int num_splits, void *workspace, size_t workspace_bytes,
+                      uint8_t *tile_status, int32_t *d_status, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSATTN_H_ */

@@ -1,0 +1,104 @@
+"""The C-ABI library loads, exports every entry point include/bsattn.h
+declares, and rejects bad arguments on the host before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bsattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_attention_bsattn_b200 import build
+    path = build.build()
+    from block_sparse_attention_bsattn_b200 import ops
+    assert os.path.samefile(ops.LIB_PATH, path)
+    return ops._lib
+
+
+def declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bsattn_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = declared()
+    for n in ("bsattn_build_index", "bsattn_fwd_prefill", "bsattn_fwd_decode",
+              "bsattn_decode_workspace_size", "bsattn_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in declared():
+        getattr(lib, n)          # AttributeError if missing
+
+
+def test_status_strings(lib):
+    from block_sparse_attention_bsattn_b200 import ops
+    assert ops.bsattn_status_string(0) == "BSATTN_OK"
+    assert ops.bsattn_status_string(-6) == "BSATTN_ERR_DEVICE_TIMEOUT"
+    assert ops.bsattn_status_string(123) == "BSATTN_UNKNOWN_STATUS"
+    assert ops.bsattn_version() >= 100
+
+
+P = ctypes.c_void_p
+
+
+def _prefill(lib, q=0x1000, k=0x2000, v=0x3000, o=0x4000, B=1, Hq=2, Hkv=2, N=256, d=128,
+             block=128, scale=0.1, causal=0, lam=0.0, rp=None, ci=None, mh=1):
+    return lib.bsattn_fwd_prefill(P(q) if q else None, P(k) if k else None, P(v) if v else None,
+                                  P(o) if o else None, None, B, Hq, Hkv, N, d, block, scale,
+                                  causal, lam, P(rp) if rp else None, P(ci) if ci else None, mh,
+                                  None, None, None)
+
+
+def test_prefill_host_validation(lib):
+    assert _prefill(lib, q=0) == -1                  # null pointer
+    assert _prefill(lib, Hq=3, Hkv=2) == -1          # Hq % Hkv
+    assert _prefill(lib, lam=1.5) == -1              # lambda outside [0, 1]
+    assert _prefill(lib, lam=float("nan")) == -1
+    assert _prefill(lib, lam=-0.1) == -1
+    assert _prefill(lib, scale=0.0) == -1
+    assert _prefill(lib, rp=0x5000, ci=None) == -1   # CSR without col_idx
+    assert _prefill(lib, rp=0x5000, ci=0x6000, mh=3) == -1
+    assert _prefill(lib, d=96) == -2                 # unsupported head dim
+    assert _prefill(lib, block=32) == -2
+    assert _prefill(lib, q=0x1001) == -3             # misaligned
+    assert _prefill(lib, o=0x4008) == -3
+
+
+def test_decode_host_validation(lib):
+    ws = lib.bsattn_decode_workspace_size(64, 32, 128, 16)
+    assert ws == 64 * 32 * 16 * (128 + 2) * 4
+
+    def dec(q=0x1000, B=2, Hq=8, Hkv=2, L=1000, d=128, block=128, lam=0.0, splits=4,
+            ws=0x9000, wsb=1 << 30):
+        return lib.bsattn_fwd_decode(P(q) if q else None, P(0x2000), P(0x3000), P(0x4000), None,
+                                     B, Hq, Hkv, L, d, block, 0.1, 0, lam, splits,
+                                     P(ws) if ws else None, wsb, None, None, None)
+    assert dec(q=0) == -1
+    assert dec(ws=0) == -1
+    assert dec(splits=0) == -1
+    assert dec(lam=2.0) == -1
+    assert dec(Hq=32, Hkv=2) == -2                   # GQA group of 16
+    assert dec(d=80) == -2
+    assert dec(q=0x1004) == -3
+    assert dec(wsb=16) == -4                         # workspace too small
+
+
+def test_index_host_validation(lib):
+    f = lib.bsattn_build_index
+    assert f(None, 1, 4, 4, 64, 64, 0, P(0x1000), P(0x2000), 16, P(0x3000), None, None) == -1
+    assert f(P(0x10), 0, 4, 4, 64, 64, 0, P(0x1000), P(0x2000), 16, P(0x3000), None, None) == -1
+    assert f(P(0x10), 1, 4, 4, 64, 64, 0, P(0x1000), P(0x2000), -1, P(0x3000), None, None) == -1
+    assert f(P(0x10), 4096, 4096, 4096, 64, 64, 0, P(0x1000), P(0x2000), 16, P(0x3000), None,
+             None) == -2
+
+
+def test_debug_hook_validation(lib):
+    assert lib.bsattn_debug_set(0, 0) == -1
+    assert lib.bsattn_debug_set(2_000_000_000, 0) == 0

@@ -1,0 +1,80 @@
+"""Decode parity: bsattn_fwd_decode (split kernel + combine, through the C ABI)
+against the fp64 oracle on the same seeded inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_bsattn_b200 import inputs
+from tests.parity import compare_outputs, compare_status
+
+pytestmark = pytest.mark.gpu
+
+
+def _ops():
+    from block_sparse_attention_bsattn_b200 import ops
+    return ops
+
+
+def _run(q, k, v, block, splits, scale, lam):
+    ops = _ops()
+    B, Hq, d = q.shape
+    Hkv, L = k.shape[1], k.shape[2]
+    T = -(-L // block)
+    st = torch.zeros(B, Hkv, T, dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = ops.bsattn_fwd_decode(q.cuda(), k.cuda(), v.cuda(), block, splits, scale, lam,
+                                   tile_status=st, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, ops.bsattn_status_string(status.item())
+    return o, lse, st
+
+
+def _check(q, k, v, block, splits, scale, lam, pairs=None, what=""):
+    o, lse, st = _run(q, k, v, block, splits, scale, lam)
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    g = Hq // Hkv
+    if pairs is None:
+        pairs = [(b, h) for b in range(B) for h in range(Hkv)]
+    qs, ks, vs = oracle.decode_problems(q, k, v, pairs)
+    ref = oracle.decode(qs.cpu(), ks.cpu(), vs.cpu(), block, scale, lam, splits)
+    o_c, lse_c, st_c = o.float().cpu().numpy(), lse.cpu().numpy(), st.cpu().numpy()
+    for p, (b, kvh) in enumerate(pairs):
+        compare_outputs(o_c[b, kvh * g:(kvh + 1) * g], ref["o"][p], lse_c[b, kvh * g:(kvh + 1) * g],
+                        ref["lse"][p], f"{what} pair {(b, kvh)}")
+        compare_status(st_c[b, kvh], ref["status"][p], ref["margin"][p], f"{what} pair {(b, kvh)}")
+    return ref
+
+
+@pytest.mark.parametrize("a", inputs.A_SWEEP)
+def test_blasst_decode_shrunk(a):
+    w = inputs.workload("blasst_decode", shrink=True)
+    _check(w.q, w.k, w.v, w.block, w.num_splits, w.scale, inputs.lambda_for(a, w.N), what=f"a={a}")
+
+
+@pytest.mark.parametrize("d,block,g", [(64, 64, 1), (64, 128, 2), (128, 64, 8), (128, 128, 4),
+                                       (128, 128, 8)])
+@pytest.mark.parametrize("splits", [1, 3, 7])
+def test_decode_shapes(d, block, g, splits):
+    B, Hkv, L = 2, 2, 5 * block + 19
+    q, k, v = inputs.blasst_decode_qkv(B, Hkv * g, Hkv, L, d, "cpu", 31 + d + g)
+    _check(q, k, v, block, splits, 1 / math.sqrt(d), 2e-3, what=f"d{d} b{block} g{g} s{splits}")
+
+
+def test_more_splits_than_tiles():
+    q, k, v = inputs.blasst_decode_qkv(1, 4, 1, 300, 128, "cpu", 9)
+    _check(q, k, v, 128, 8, 1 / math.sqrt(128), 1e-2, what="empty splits")
+
+
+@pytest.mark.parametrize("a", [0.0, 10.0])
+def test_blasst_decode_full_size_sampled(a):
+    """B64 Hq32/Hkv8 L131072 d128, 16 splits, in the launch configuration the
+    benchmark times; 8 (batch, KV head) problems checked against the oracle."""
+    w = inputs.workload("blasst_decode", device="cuda")
+    rng = np.random.default_rng(17)
+    pairs = sorted({(int(rng.integers(w.B)), int(rng.integers(w.Hkv))) for _ in range(8)})
+    _check(w.q, w.k, w.v, w.block, w.num_splits, w.scale, inputs.lambda_for(a, w.N), pairs,
+           what=f"full a={a}")

@@ -1,0 +1,156 @@
+"""Prefill parity: the CUDA path (bsattn_build_index + bsattn_fwd_prefill
+through the C ABI) against the fp64 oracle on the same seeded inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_bsattn_b200 import inputs
+from tests.parity import compare_outputs, compare_status
+
+pytestmark = pytest.mark.gpu
+
+
+def _ops():
+    from block_sparse_attention_bsattn_b200 import ops
+    return ops
+
+
+def _run_gpu(w, lam, mask=None, mask_heads=1):
+    ops = _ops()
+    q, k, v = w.q.cuda(), w.k.cuda(), w.v.cuda()
+    rp = ci = None
+    if mask is not None:
+        m = torch.as_tensor(mask, dtype=torch.uint8).cuda().contiguous()
+        rp, ci, _ = ops.bsattn_build_index(m, w.block, w.block, w.causal)
+        mask_heads = m.shape[0]
+    st = torch.zeros(w.B, w.Hq, w.nq, w.nk, dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = ops.bsattn_fwd_prefill(q, k, v, w.block, w.scale, w.causal, lam, rp, ci, mask_heads,
+                                    tile_status=st, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0, ops.bsattn_status_string(status.item())
+    return o, lse, st
+
+
+def _check(w, lam, mask=None, what=""):
+    o, lse, st = _run_gpu(w, lam, mask)
+    ref = oracle.prefill(w.q, w.k, w.v, w.block, w.scale, w.causal, lam, mask=mask)
+    compare_outputs(o, ref["o"], lse, ref["lse"], what)
+    compare_status(st, ref["status"], ref["margin"], what)
+    return ref
+
+
+@pytest.mark.parametrize("name", ["tiny", "mmdit", "videodit"])
+def test_static_mask_workloads_shrunk(name):
+    w = inputs.workload(name, shrink=True)
+    _check(w, 0.0, w.mask.numpy(), name)
+
+
+def test_mmdit_full_size():
+    """Multimodal DiT at full size (B1 H24 N4352 d64 block 128): every output."""
+    w = inputs.workload("mmdit")
+    _check(w, 0.0, w.mask.numpy(), "mmdit")
+
+
+@pytest.mark.parametrize("a", inputs.A_SWEEP)
+def test_blasst_prefill_shrunk(a):
+    w = inputs.workload("blasst_prefill", shrink=True)
+    ref = _check(w, inputs.lambda_for(a, w.N), None, f"blasst a={a}")
+    if a >= 10:
+        assert (ref["status"] == 1).sum() > 0
+
+
+@pytest.mark.parametrize("d,block", [(64, 64), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_dense_shapes_and_tails(d, block, causal):
+    """Every (d, block) variant, causal and not, with a ragged tail and GQA 4."""
+    B, Hq, Hkv, N = 2, 4, 1, 3 * block + 37
+    q, k, v = inputs.normal_qkv(B, Hq, Hkv, N, d, "cpu", 100 + d + block)
+    w = inputs.Workload("dense", B, Hq, Hkv, N, d, block, causal, "prefill", 1 / math.sqrt(d),
+                        None, q=q, k=k, v=v)
+    _check(w, 0.0, None, f"d{d} b{block} c{causal}")
+
+
+@pytest.mark.parametrize("d,block", [(64, 64), (128, 128)])
+def test_blasst_random_masks_per_head(d, block):
+    """Per-head random static masks combined with the dynamic skip."""
+    rng = np.random.default_rng(d + block)
+    B, Hq, Hkv, N = 1, 4, 2, 6 * block - 5
+    nb = -(-N // block)
+    m = (rng.random((Hq, nb, nb)) < 0.6).astype(np.uint8)
+    m[:, np.arange(nb), np.arange(nb)] = 1
+    m[:, 2, :] = 0                                 # an empty row
+    q, k, v = inputs.blasst_prefill_qkv(B, Hq, Hkv, N, d, "cpu", 7)
+    w = inputs.Workload("rand", B, Hq, Hkv, N, d, block, True, "prefill", 1 / math.sqrt(d), None,
+                        q=q, k=k, v=v)
+    o, lse, st = _run_gpu(w, 3e-3, m)
+    ref = oracle.prefill(q, k, v, block, w.scale, True, 3e-3, mask=m)
+    compare_outputs(o, ref["o"], lse, ref["lse"])
+    compare_status(st, ref["status"], ref["margin"])
+    # the empty row: zeros and -inf
+    rows = slice(2 * block, 3 * block)
+    assert (o[:, :, rows].float() == 0).all()
+    assert torch.isneginf(lse[:, :, rows]).all()
+
+
+def test_short_sequence_single_partial_tile():
+    q, k, v = inputs.normal_qkv(1, 2, 2, 50, 128, "cpu", 3)
+    w = inputs.Workload("short", 1, 2, 2, 50, 128, 128, True, "prefill", 1 / math.sqrt(128), None,
+                        q=q, k=k, v=v)
+    _check(w, 0.5, None, "short")
+
+
+def test_closed_form_skip_on_gpu():
+    """The two-tile closed form of the oracle pins, on the GPU (block 64, d 64)."""
+    N, d = 128, 64
+    qn = np.zeros((N, d)); qn[:, 0] = 1.0
+    kn = np.zeros((N, d)); kn[0, 0] = 10.0; kn[64:, 0] = 2.0
+    vn = np.round(np.random.default_rng(0).standard_normal((N, d)) * 8) / 8
+    t = lambda x: torch.tensor(x, dtype=torch.float32).to(torch.bfloat16)[None, None].contiguous()
+    w = inputs.Workload("cf", 1, 1, 1, N, d, 64, False, "prefill", 1.0, None, q=t(qn), k=t(kn), v=t(vn))
+    o, lse, st = _run_gpu(w, math.exp(-5))
+    assert (st[0, 0, :, 1] == 1).all() and (st[0, 0, :, 0] == 2).all()
+    expect = (math.exp(10) * vn[0] + vn[1:64].sum(0)) / (math.exp(10) + 63)
+    assert np.abs(o[0, 0].float().cpu().numpy() - expect[None]).max() < 2e-2
+
+
+def _sampled_items(w, n_items, seed):
+    rng = np.random.default_rng(seed)
+    items = set()
+    # always include the first and the last query tile of some heads
+    for h in rng.choice(w.Hq, size=min(2, w.Hq), replace=False):
+        items.add((0, int(h), 0))
+        items.add((0, int(h), w.nq - 1))
+    while len(items) < n_items:
+        items.add((int(rng.integers(w.B)), int(rng.integers(w.Hq)), int(rng.integers(w.nq))))
+    return sorted(items)
+
+
+def _check_sampled(w, lam, mask, n_items, what):
+    """Full-size workload in the launch configuration the benchmark times,
+    compared on sampled query tiles that the oracle computes one by one."""
+    o, lse, st = _run_gpu(w, lam, mask)
+    items = _sampled_items(w, n_items, 5)
+    ref = oracle.prefill(w.q.cpu(), w.k.cpu(), w.v.cpu(), w.block, w.scale, w.causal, lam,
+                         mask=mask, items=items)
+    o_c, lse_c, st_c = o.float().cpu().numpy(), lse.cpu().numpy(), st.cpu().numpy()
+    for (b, h, i) in items:
+        rows = slice(i * w.block, min(w.N, (i + 1) * w.block))
+        compare_outputs(o_c[b, h, rows], ref["o"][b, h, rows], lse_c[b, h, rows],
+                        ref["lse"][b, h, rows], f"{what} item {(b, h, i)}")
+        compare_status(st_c[b, h, i], ref["status"][b, h, i], ref["margin"][b, h, i],
+                       f"{what} item {(b, h, i)}")
+
+
+def test_videodit_full_size_sampled():
+    w = inputs.workload("videodit", device="cuda")
+    _check_sampled(w, 0.0, w.mask.numpy(), 24, "videodit")
+
+
+@pytest.mark.parametrize("a", [0.0, 10.0])
+def test_blasst_prefill_full_size_sampled(a):
+    w = inputs.workload("blasst_prefill", device="cuda")
+    _check_sampled(w, inputs.lambda_for(a, w.N), None, 24, f"blasst a={a}")
