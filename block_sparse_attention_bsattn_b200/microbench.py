@@ -1,0 +1,97 @@
+"""Time one entry point of the library on a chosen slice of a workload.
+
+    python -m block_sparse_attention_bsattn_b200.microbench prefill --heads 8 --n 8192 --a 10
+    python -m block_sparse_attention_bsattn_b200.microbench decode --batch 8 --a 10
+    python -m block_sparse_attention_bsattn_b200.microbench videodit --heads 4
+
+Used for Nsight Compute captures of a single kernel on a small case (a few
+launches, a few hundred MB on the device) and for quick CUDA-event timings.
+Prints one JSON line with the per-launch time and the algorithmic work.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import torch
+
+from . import inputs, ops
+
+TILE = 2 * 128 * 128 * 128
+
+
+def _time(fn, iters):
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(iters):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / iters
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("what", choices=("prefill", "decode", "videodit", "mmdit"))
+    ap.add_argument("--heads", type=int, default=8, help="query heads (prefill/videodit/mmdit)")
+    ap.add_argument("--n", type=int, default=32768, help="sequence length (prefill)")
+    ap.add_argument("--batch", type=int, default=64, help="batch (decode)")
+    ap.add_argument("--l", type=int, default=131072, help="KV length (decode)")
+    ap.add_argument("--a", type=float, default=10.0)
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=2)
+    args = ap.parse_args()
+    torch.cuda.set_device(0)
+    out = {"what": args.what}
+    if args.what == "prefill":
+        hkv = max(1, args.heads // 4)
+        q, k, v = inputs.blasst_prefill_qkv(1, args.heads, hkv, args.n, 128, "cuda", 1237)
+        lam = inputs.lambda_for(args.a, args.n)
+        nq = args.n // 128
+        st = torch.zeros(1, args.heads, nq, nq, dtype=torch.uint8, device="cuda")
+        o, _ = ops.bsattn_fwd_prefill(q, k, v, 128, None, True, lam, tile_status=st)
+        torch.cuda.synchronize()
+        vis, exe = int((st > 0).sum()), int((st == 2).sum())
+        fn = lambda: ops.bsattn_fwd_prefill(q, k, v, 128, None, True, lam, o=o, want_lse=False)
+        for _ in range(args.warmup):
+            fn()
+        ms = _time(fn, args.iters)
+        out.update(heads=args.heads, n=args.n, a=args.a, visited=vis, executed=exe, ms=ms,
+                   tflops=TILE * (vis + exe) / ms / 1e9)
+    elif args.what in ("videodit", "mmdit"):
+        w = inputs.workload(args.what, device="cuda", generate=False)
+        q, k, v = inputs.normal_qkv(1, args.heads, args.heads, w.N, w.d, "cuda", 1236)
+        m = w.mask.cuda()
+        rp, ci, nnz = ops.bsattn_build_index(m, w.block, w.block, False)
+        fn = lambda: ops.bsattn_fwd_prefill(q, k, v, w.block, w.scale, False, 0.0, rp, ci, 1,
+                                            want_lse=False)
+        for _ in range(args.warmup):
+            fn()
+        ms = _time(fn, args.iters)
+        tiles = int(nnz.sum()) * args.heads
+        flops = 4 * w.block * w.block * w.d * tiles
+        out.update(heads=args.heads, n=w.N, d=w.d, tiles=tiles, ms=ms, tflops=flops / ms / 1e9)
+    else:
+        B, Hq, Hkv, L, d = args.batch, 32, 8, args.l, 128
+        q, k, v = inputs.blasst_decode_qkv(B, Hq, Hkv, L, d, "cuda", 1238)
+        lam = inputs.lambda_for(args.a, L)
+        T = -(-L // 128)
+        st = torch.zeros(B, Hkv, T, dtype=torch.uint8, device="cuda")
+        ws = torch.empty(ops.bsattn_decode_workspace_size(B, Hq, d, 16), dtype=torch.uint8,
+                         device="cuda")
+        o, _ = ops.bsattn_fwd_decode(q, k, v, 128, 16, None, lam, workspace=ws, tile_status=st)
+        torch.cuda.synchronize()
+        vis, exe = int((st > 0).sum()), int((st == 2).sum())
+        fn = lambda: ops.bsattn_fwd_decode(q, k, v, 128, 16, None, lam, o=o, want_lse=False,
+                                           workspace=ws)
+        for _ in range(args.warmup):
+            fn()
+        ms = _time(fn, args.iters)
+        byt = 2 * B * Hq * d * 2 + 128 * d * 2 * (vis + exe)
+        out.update(batch=B, l=L, a=args.a, visited=vis, executed=exe, ms=ms, gbs=byt / ms / 1e6)
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

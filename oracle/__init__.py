@@ -49,23 +49,27 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def bind(lib: ctypes.CDLL) -> ctypes.CDLL:
+    """Declare the C signatures on a loaded oracle library."""
+    P = ctypes.c_void_p
+    i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+    lib.oracle_build_index.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, i64, P]
+    lib.oracle_build_index.restype = i32
+    lib.oracle_prefill.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, i32,
+                                   f64, P, i32, P, i32, P, P, P, P]
+    lib.oracle_prefill.restype = i32
+    lib.oracle_decode.argtypes = [P, P, P, i32, i32, i64, i32, i32, f64, f64, i32,
+                                  P, P, P, P]
+    lib.oracle_decode.restype = i32
+    lib.oracle_num_threads.restype = i32
+    return lib
+
+
 def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
-            P = ctypes.c_void_p
-            i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
-            lib.oracle_build_index.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, i64, P]
-            lib.oracle_build_index.restype = i32
-            lib.oracle_prefill.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, i32,
-                                           f64, P, i32, P, i32, P, P, P, P]
-            lib.oracle_prefill.restype = i32
-            lib.oracle_decode.argtypes = [P, P, P, i32, i32, i64, i32, i32, f64, f64, i32,
-                                          P, P, P, P]
-            lib.oracle_decode.restype = i32
-            lib.oracle_num_threads.restype = i32
-            _lib = lib
+            _lib = bind(ctypes.CDLL(build()))
     return _lib
 
 
