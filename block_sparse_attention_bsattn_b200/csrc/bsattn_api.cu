@@ -19,6 +19,8 @@ namespace bsattn {
 // ------------------------------------------------------------------ debug knobs
 static unsigned long long g_wait_limit_ns = 2000000000ull;  // 2 s
 static int g_inject_stall = 0;
+static volatile int32_t* g_trace = nullptr;
+static int g_trace_n = 0;
 
 // ------------------------------------------------------------------ driver entry
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -97,6 +99,35 @@ int bsattn_debug_set(long long wait_limit_ns, int inject_stall) {
   return BSATTN_OK;
 }
 
+int bsattn_debug_trace(int n, int32_t** host_view) {
+  static int32_t* host_buf = nullptr;
+  if (n < 0 || (n > 0 && !host_view)) return BSATTN_ERR_INVALID_ARG;
+  g_trace = nullptr;
+  g_trace_n = 0;
+  if (host_buf) {
+    cudaFreeHost(host_buf);
+    host_buf = nullptr;
+  }
+  if (n == 0) {
+    if (host_view) *host_view = nullptr;
+    return BSATTN_OK;
+  }
+  if (cudaHostAlloc(reinterpret_cast<void**>(&host_buf), sizeof(int32_t) * (size_t)n,
+                    cudaHostAllocMapped) != cudaSuccess)
+    return BSATTN_ERR_CUDA;
+  std::memset(host_buf, 0, sizeof(int32_t) * (size_t)n);
+  void* dev = nullptr;
+  if (cudaHostGetDevicePointer(&dev, host_buf, 0) != cudaSuccess) {
+    cudaFreeHost(host_buf);
+    host_buf = nullptr;
+    return BSATTN_ERR_CUDA;
+  }
+  g_trace = static_cast<volatile int32_t*>(dev);
+  g_trace_n = n;
+  *host_view = host_buf;
+  return BSATTN_OK;
+}
+
 int bsattn_build_index(const uint8_t* d_mask, int mask_heads, int nq_blocks, int nk_blocks,
                        int q_block, int k_block, int causal, int32_t* d_row_ptr,
                        int32_t* d_col_idx, int64_t col_capacity, int32_t* d_nnz,
@@ -162,6 +193,8 @@ int bsattn_fwd_prefill(const void* q, const void* k, const void* v, void* o, flo
   p.thr_log2 = lambda > 0.f ? (float)std::log2((double)lambda) : -INFINITY;
   p.debug_stall = g_inject_stall;
   p.wait_limit_ns = g_wait_limit_ns;
+  p.trace = g_trace;
+  p.trace_n = g_trace_n;
 
   cudaError_t e;
   if (d == 128 && block == 128) e = launch_prefill<128, 128>(tq, tk, tv, p, (int)items, stream);
@@ -226,6 +259,8 @@ int bsattn_fwd_decode(const void* q, const void* k, const void* v, void* o, floa
   p.use_skip = lambda > 0.f ? 1 : 0;
   p.thr_log2 = lambda > 0.f ? (float)std::log2((double)lambda) : -INFINITY;
   p.wait_limit_ns = g_wait_limit_ns;
+  p.trace = g_trace;
+  p.trace_n = g_trace_n;
 
   cudaError_t e = cudaErrorInvalidValue;
 #define BSATTN_DEC(DD, BB, GG)                                               \

@@ -31,6 +31,8 @@ struct PrefillParams {
   int use_skip;      // lambda > 0
   int debug_stall;   // test hook: the producer never issues the Q load
   unsigned long long wait_limit_ns;
+  volatile int32_t* trace;  // debug: progress markers (host-visible memory) or null
+  int trace_n;
 };
 
 struct DecodeParams {
@@ -45,6 +47,8 @@ struct DecodeParams {
   float thr_log2;
   int use_skip;
   unsigned long long wait_limit_ns;
+  volatile int32_t* trace;
+  int trace_n;
 };
 
 struct CombineParams {

@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(256, 1)
   const int nt = max(0, t_end - t_begin);
   const int zc = b * p.Hkv + kvh;
 
+  if (tid == 0) trace_mark(p.trace, p.trace_n, 16 + blockIdx.x, 1);
   if (tid == 0) {
     for (int s = 0; s < C::KST; ++s) mbar_init(&bars->k_full[s], 1);
     for (int s = 0; s < C::VST; ++s) mbar_init(&bars->v_full[s], 1);
@@ -317,6 +318,7 @@ __global__ void __launch_bounds__(256, 1)
       for (int k = max(0, issued_v - C::VST); k < issued_v; ++k)
         mbar_wait_drain(&bars->v_full[k % C::VST], (k / C::VST) & 1, lim);
       report_status(p.status, kDevTimeout);
+      trace_mark(p.trace, p.trace_n, 16 + blockIdx.x, 13);
     }
     return;
   }
@@ -356,6 +358,7 @@ __global__ void __launch_bounds__(256, 1)
     p.ws_l[base + (int64_t)tid * p.splits] = kept_total > 0 ? s : 0.f;
     p.ws_m[base + (int64_t)tid * p.splits] = kept_total > 0 ? m_ref[tid] : -INFINITY;
   }
+  if (tid == 0) trace_mark(p.trace, p.trace_n, 16 + blockIdx.x, 3);
 }
 
 // One CTA per (batch, query head), one thread per output dimension.

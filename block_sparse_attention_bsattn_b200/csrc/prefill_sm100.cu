@@ -123,6 +123,10 @@ __global__ void __launch_bounds__(192, 1)
     n = p.causal ? i + 1 : p.nk;
   }
 
+  // debug trace: slot 16 + CTA = stage reached; CTA 0 also records per-role progress
+  const bool tr0 = blockIdx.x == 0;
+  if (threadIdx.x == 0) trace_mark(p.trace, p.trace_n, 16 + blockIdx.x, 1);
+
   // ---- setup
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -150,6 +154,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const uint64_t lim = p.wait_limit_ns;
+  if (threadIdx.x == 0) trace_mark(p.trace, p.trace_n, 16 + blockIdx.x, 2);
 
   if (warp == 0) {
     // ======================================================== TMA producer
@@ -180,7 +185,9 @@ __global__ void __launch_bounds__(192, 1)
           tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
                       hf * 64, j * BLK, b * p.Hkv + kvh);
         ++issued_v;
+        if (tr0) trace_mark(p.trace, p.trace_n, 1, t + 1);
       }
+      if (tr0) trace_mark(p.trace, p.trace_n, 1, 100000 + issued_k);
       if (*abort) {
         // let every copy this thread started land before the CTA can exit
         for (int t = (issued_k > C::KST ? issued_k - C::KST : 0); t < issued_k; ++t)
@@ -242,10 +249,13 @@ __global__ void __launch_bounds__(192, 1)
         } else {
           mbar_arrive(&bars->v_empty[vs]);
         }
+        if (tr0) trace_mark(p.trace, p.trace_n, 2, t + 1);
       }
+      if (tr0) trace_mark(p.trace, p.trace_n, 2, 100000 + kept);
       // all tcgen05 work issued by this thread must finish before TMEM is freed
       mma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0, lim);
+      if (tr0) trace_mark(p.trace, p.trace_n, 3, 1);
     }
   } else {
     // ======================================================== softmax warps
@@ -315,27 +325,17 @@ __global__ void __launch_bounds__(192, 1)
           if (!mbar_wait(&bars->o_done, (kept - 1) & 1, abort, lim)) { ok = false; break; }
           tc_fence_after();
         }
-        float m_new = m_ref;
+        // exponent shift: set by the first kept tile, then moved only when the
+        // running max exceeds it by more than TAU (O and l rescaled below)
+        float alpha = 1.f;
+        bool rescale = false;
         if (kept == 0) {
-          m_new = m_run;
+          m_ref = m_run;
         } else if (m_run > m_ref + C::TAU) {
-          m_new = m_run;
-          const float alpha = fast_exp2(m_ref - m_new);
-          l *= alpha;
-          if (in_tile) {
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t r[32];
-              tmem_ld32(lane_addr + C::O_COL + c0, r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-              tmem_st32(lane_addr + C::O_COL + c0, r);
-            }
-            tmem_wait_st();
-          }
+          alpha = fast_exp2(m_ref - m_run);
+          rescale = true;
+          m_ref = m_run;
         }
-        m_ref = m_new;
         const float shift = (m_ref == -INFINITY) ? 0.f : m_ref;
         if (in_tile) {
           float rs = 0.f;
@@ -351,8 +351,20 @@ __global__ void __launch_bounds__(192, 1)
             }
             tmem_st16(lane_addr + C::S_COL + sb * 128 + c0 / 2, pk);
           }
+          l = l * alpha + rs;
+          // rare: bring the accumulated O to the new shift (no BMM2 is in flight)
+          if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t r[32];
+              tmem_ld32(lane_addr + C::O_COL + c0, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+              tmem_st32(lane_addr + C::O_COL + c0, r);
+            }
+          }
           tmem_wait_st();
-          l += rs;
         }
         ++kept;
       }
@@ -360,6 +372,7 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready[sb]);
+      if (tr0 && lane == 0) trace_mark(p.trace, p.trace_n, 4 + sw, t + 1);
     }
 
     // ---- epilogue: O / l -> bf16, LSE
@@ -396,12 +409,15 @@ __global__ void __launch_bounds__(192, 1)
   }
 
   // ---- teardown
+  if (lane == 0) trace_mark(p.trace, p.trace_n, tr0 ? 8 + warp : p.trace_n, 1);
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) trace_mark(p.trace, p.trace_n, 16 + blockIdx.x, bars->abort ? 13 : 3);
   if (threadIdx.x == 0 && bars->abort) report_status(p.status, kDevTimeout);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+    if (lane == 0) trace_mark(p.trace, p.trace_n, 16 + blockIdx.x, bars->abort ? 14 : 4);
   }
 }
 

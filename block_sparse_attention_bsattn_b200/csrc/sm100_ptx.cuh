@@ -250,6 +250,16 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Debug progress marker: slot `i` of a host-visible trace buffer (no-op when
+// tracing is off).  Stores are volatile and fenced at system scope so that a
+// host thread can watch them while the kernel runs.
+__device__ __forceinline__ void trace_mark(volatile int32_t* trace, int n, int i, int32_t v) {
+  if (trace && i < n) {
+    trace[i] = v;
+    __threadfence_system();
+  }
+}
+
 __device__ __forceinline__ void report_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, 0, code);
 }

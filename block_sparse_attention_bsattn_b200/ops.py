@@ -35,6 +35,8 @@ _lib.bsattn_status_string.restype = ctypes.c_char_p
 _lib.bsattn_version.restype = _I
 _lib.bsattn_debug_set.argtypes = [ctypes.c_longlong, _I]
 _lib.bsattn_debug_set.restype = _I
+_lib.bsattn_debug_trace.argtypes = [_I, ctypes.POINTER(ctypes.POINTER(ctypes.c_int32))]
+_lib.bsattn_debug_trace.restype = _I
 _lib.bsattn_build_index.argtypes = [_P, _I, _I, _I, _I, _I, _I, _P, _P, _I64, _P, _P, _P]
 _lib.bsattn_build_index.restype = _I
 _lib.bsattn_fwd_prefill.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F,
@@ -46,7 +48,8 @@ _lib.bsattn_fwd_decode.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _
                                    _P, _SZ, _P, _P, _P]
 _lib.bsattn_fwd_decode.restype = _I
 
-EXPORTED = ("bsattn_status_string", "bsattn_version", "bsattn_debug_set", "bsattn_build_index",
+EXPORTED = ("bsattn_status_string", "bsattn_version", "bsattn_debug_set", "bsattn_debug_trace",
+            "bsattn_build_index",
             "bsattn_fwd_prefill", "bsattn_decode_workspace_size", "bsattn_fwd_decode")
 
 
@@ -70,6 +73,18 @@ def bsattn_debug_set(wait_limit_ns: int = 2_000_000_000, inject_stall: bool = Fa
     rc = _lib.bsattn_debug_set(int(wait_limit_ns), int(bool(inject_stall)))
     if rc:
         raise BsattnError(rc, "bsattn_debug_set")
+
+
+def bsattn_debug_trace(n: int):
+    """Debugging aid: n > 0 makes the kernels record progress markers into a
+    library-owned mapped host buffer of n int32 and returns a numpy view of it
+    (readable while a kernel runs); n = 0 turns tracing off and returns None."""
+    import numpy as np
+    view = ctypes.POINTER(ctypes.c_int32)()
+    rc = _lib.bsattn_debug_trace(int(n), ctypes.byref(view))
+    if rc:
+        raise BsattnError(rc, "bsattn_debug_trace")
+    return np.ctypeslib.as_array(view, shape=(n,)) if n > 0 else None
 
 
 def _ptr(t: Optional[torch.Tensor]):

@@ -71,6 +71,19 @@ int bsattn_version(void);
 int bsattn_debug_set(long long wait_limit_ns, int inject_stall);
 
 /*
+ * bsattn_debug_trace -- debugging aid, process-wide.  n > 0 allocates n int32
+ * of mapped, pinned host memory (zeroed; the only allocation the library ever
+ * makes, and on the host), returns its host address in *host_view and makes
+ * the prefill and decode kernels record progress there, readable while a
+ * kernel is still running: slot 16 + CTA index holds the stage a CTA reached
+ * (1 entered, 2 set up, 3 finished, 4 tensor memory freed; 13/14 the same
+ * after a timed-out wait), slots 1..11 the per-role progress of CTA 0.  n = 0
+ * frees the buffer and turns tracing off.  Negative n or a NULL host_view
+ * with n > 0 give BSATTN_ERR_INVALID_ARG.
+ */
+int bsattn_debug_trace(int n, int32_t **host_view);
+
+/*
  * bsattn_build_index -- block mask -> per-query-block CSR lists.
  *
  * Follows "块稀疏Attention实战" section 2.3 (keep the mask as an index of its
