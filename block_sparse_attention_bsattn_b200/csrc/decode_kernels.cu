@@ -170,7 +170,9 @@ __global__ void __launch_bounds__(256, 1)
     if (it < nt) {
       const int t = it;
       const int ks = t % C::KST;
-      bool failed = !mbar_wait(&bars->k_full[ks], (t / C::KST) & 1, abort, lim);
+      // warp-uniform outcome: the shuffles below need every lane
+      const bool failed =
+          __any_sync(0xffffffffu, !mbar_wait(&bars->k_full[ks], (t / C::KST) & 1, abort, lim));
       float acc[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) acc[g] = 0.f;
@@ -278,7 +280,8 @@ __global__ void __launch_bounds__(256, 1)
       const int kidx = kept_total - 1 - __popc(hist & ((1u << C::LA) - 1u));
       const int slot = kidx % C::VST;
       const int vphase = (kidx / C::VST) & 1;
-      bool failed = !mbar_wait(&bars->v_full[slot], vphase, abort, lim);
+      const bool failed =
+          __any_sync(0xffffffffu, !mbar_wait(&bars->v_full[slot], vphase, abort, lim));
       if (!failed && tid < BLK) {
         float pr[G];
 #pragma unroll

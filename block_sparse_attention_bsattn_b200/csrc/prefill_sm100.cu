@@ -272,7 +272,10 @@ __global__ void __launch_bounds__(192, 1)
     for (int t = 0; t < n; ++t) {
       const int j = cols ? cols[t] : t;
       const int sb = t & 1;
-      if (!mbar_wait(&bars->s_full[sb], (t >> 1) & 1, abort, lim)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (t >> 1) & 1, abort, lim))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       float s[BLK];
       if (in_tile) {
@@ -311,7 +314,11 @@ __global__ void __launch_bounds__(192, 1)
           mbar_arrive(&bars->vote_bar[t & 1]);
         }
         __syncwarp();
-        if (!mbar_wait(&bars->vote_bar[t & 1], (t >> 1) & 1, abort, lim)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&bars->vote_bar[t & 1], (t >> 1) & 1, abort, lim))) {
+          ok = false;
+          break;
+        }
         volatile int* vv = bars->vote[t & 1];
         skip = vv[0] & vv[1] & vv[2] & vv[3];
       }
@@ -322,7 +329,10 @@ __global__ void __launch_bounds__(192, 1)
         if (kept > 0) {
           // the previous BMM2 must be complete before P overwrites this S
           // buffer's neighbour state and before O may be rescaled
-          if (!mbar_wait(&bars->o_done, (kept - 1) & 1, abort, lim)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (kept - 1) & 1, abort, lim))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
         }
         // exponent shift: set by the first kept tile, then moved only when the
@@ -375,12 +385,15 @@ __global__ void __launch_bounds__(192, 1)
       if (tr0 && lane == 0) trace_mark(p.trace, p.trace_n, 4 + sw, t + 1);
     }
 
-    // ---- epilogue: O / l -> bf16, LSE
+    // ---- epilogue: O / l -> bf16, LSE.  tcgen05.ld is warp-collective, so
+    // every lane of a warp that owns tile rows loads; only rows inside the
+    // sequence are stored.
     if (ok && kept > 0) {
-      if (!mbar_wait(&bars->o_done, (kept - 1) & 1, abort, lim)) ok = false;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (kept - 1) & 1, abort, lim)))
+        ok = false;
       tc_fence_after();
     }
-    if (ok && valid) {
+    if (ok && in_tile) {
       const int64_t orow = ((int64_t)b * p.Hq + h) * p.N + r0 + row;
       __nv_bfloat16* dst = p.o + orow * D;
       const bool have = kept > 0 && l > 0.f;
@@ -392,19 +405,22 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld32(lane_addr + C::O_COL + c0, r);
           tmem_wait_ld();
         }
-        uint32_t w[16];
+        if (valid) {
+          uint32_t w[16];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float a0 = have ? __uint_as_float(r[c]) * inv_l : 0.f;
-          const float a1 = have ? __uint_as_float(r[c + 1]) * inv_l : 0.f;
-          w[c / 2] = pack_bf16x2(a0, a1);
+          for (int c = 0; c < 32; c += 2) {
+            const float a0 = have ? __uint_as_float(r[c]) * inv_l : 0.f;
+            const float a1 = have ? __uint_as_float(r[c + 1]) * inv_l : 0.f;
+            w[c / 2] = pack_bf16x2(a0, a1);
+          }
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
-        uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
       }
-      if (p.lse) p.lse[orow] = have ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      if (valid && p.lse)
+        p.lse[orow] = have ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
 
