@@ -24,7 +24,8 @@ def compare_outputs(o_gpu, ref_o, lse_gpu=None, ref_lse=None, what=""):
     if lse_gpu is not None:
         lse = lse_gpu.float().cpu().numpy() if isinstance(lse_gpu, torch.Tensor) else lse_gpu
         both_inf = np.isneginf(lse) & np.isneginf(ref_lse)
-        d = np.where(both_inf, 0.0, np.abs(lse - ref_lse))
+        with np.errstate(invalid="ignore"):
+            d = np.where(both_inf, 0.0, np.abs(lse - ref_lse))
         assert np.nanmax(d) <= LSE_MAX_ABS, f"{what}: lse max-abs {np.nanmax(d):.3e}"
     return float(err.max()), float(err.mean())
 
