@@ -47,10 +47,14 @@ _lib.bsattn_decode_workspace_size.restype = _SZ
 _lib.bsattn_fwd_decode.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F, _I,
                                    _P, _SZ, _P, _P, _P]
 _lib.bsattn_fwd_decode.restype = _I
+_lib.bsattn_fwd_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I,
+                                           _F, _I, _P, _P, _P]
+_lib.bsattn_fwd_decode_noalloc.restype = _I
 
 EXPORTED = ("bsattn_status_string", "bsattn_version", "bsattn_debug_set", "bsattn_debug_trace",
             "bsattn_build_index",
-            "bsattn_fwd_prefill", "bsattn_decode_workspace_size", "bsattn_fwd_decode")
+            "bsattn_fwd_prefill", "bsattn_decode_workspace_size", "bsattn_fwd_decode",
+            "bsattn_fwd_decode_noalloc")
 
 
 class BsattnError(RuntimeError):
@@ -188,4 +192,31 @@ def bsattn_fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: 
                                 _ptr(tile_status), _ptr(status), _stream(stream))
     if rc:
         raise BsattnError(rc, "bsattn_fwd_decode")
+    return o, lse
+
+
+def bsattn_fwd_decode_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int,
+                              num_splits: int, o: torch.Tensor, scale: Optional[float] = None,
+                              lam: float = 0.0, lse: Optional[torch.Tensor] = None,
+                              tile_status: Optional[torch.Tensor] = None,
+                              status: Optional[torch.Tensor] = None, stream=None):
+    """Decode for callers that cannot allocate device memory: the library's
+    own 32 MiB scratch array replaces the workspace, and every output buffer
+    (o, and lse / tile_status when wanted) comes from the caller."""
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k, "k", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    _check(o, "o", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    Hkv, L = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, L, d) or v.shape != k.shape or o.shape != q.shape:
+        raise ValueError("k/v must be [B, Hkv, L, d] and o [B, Hq, d] matching q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = _lib.bsattn_fwd_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq,
+                                        Hkv, L, d, int(block), float(scale), 0, float(lam),
+                                        int(num_splits), _ptr(tile_status), _ptr(status),
+                                        _stream(stream))
+    if rc:
+        raise BsattnError(rc, "bsattn_fwd_decode_noalloc")
     return o, lse

@@ -169,6 +169,35 @@ int bsattn_fwd_decode(const void *q, const void *k, const void *v, void *o, floa
                       float lambda, int num_splits, void *workspace, size_t workspace_bytes,
                       uint8_t *tile_status, int32_t *d_status, cudaStream_t stream);
 
+/*
+ * bsattn_fwd_decode_noalloc -- bsattn_fwd_decode for callers that cannot
+ * allocate device memory.  The pages have no counterpart of this entry point.
+ *
+ * Some callers cannot call cudaMalloc at all: code inside a host framework
+ * that owns all device memory and hands extensions only their input and
+ * output buffers (an inference engine with one pre-planned memory arena, for
+ * instance), or latency-critical service paths where an allocation's cost and
+ * possible failure are not acceptable.  They cannot provide the decode
+ * workspace, so this variant uses a scratch array inside the library: a
+ * file-scope device array of 32 MiB, held on every GPU that loads the library
+ * until the process exits.  The call itself allocates nothing.
+ *
+ * Arguments, layouts and results are those of bsattn_fwd_decode without the
+ * workspace.  Problems whose split outputs need more than 32 MiB
+ * (bsattn_decode_workspace_size(B, Hq, d, num_splits) > 33554432) are rejected
+ * with BSATTN_ERR_CAPACITY before anything runs.
+ *
+ * The first call on each device (with that device current) looks up the
+ * scratch array's device address once, so make it before any stream capture.
+ * Every call shares the one scratch array, which keeps the last call's
+ * contents; no part of it needs to start at zero.  Calls whose kernels may
+ * overlap on the GPU (unordered streams) race on it and must be serialised.
+ */
+int bsattn_fwd_decode_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                              int B, int Hq, int Hkv, int L, int d, int block, float scale,
+                              int causal, float lambda, int num_splits, uint8_t *tile_status,
+                              int32_t *d_status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
