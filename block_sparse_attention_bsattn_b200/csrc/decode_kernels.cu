@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(256, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
   using C = DecodeCfg<D, BLK, G>;
+  static_assert(sizeof(DecodeBarriers) <= 128, "barrier block");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));

@@ -163,6 +163,9 @@ size_t bsattn_decode_workspace_size(int B, int Hq, int d, int num_splits);
  *   workspace   device scratch of at least bsattn_decode_workspace_size(...)
  *               bytes, 16-byte aligned, owned by the caller
  *   tile_status uint8 [B][Hkv][T] or NULL (cleared, then 1 skipped / 2 executed)
+ *
+ * Supported GQA groups Hq/Hkv: 1..16 with block 128 (tensor-core kernel),
+ * 1, 2, 4 or 8 with block 64; anything else gives BSATTN_ERR_UNSUPPORTED.
  */
 int bsattn_fwd_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B,
                       int Hq, int Hkv, int L, int d, int block, float scale, int causal,
