@@ -2,7 +2,8 @@
 """Benchmark of the block-sparse attention hot path on B200.
 
 One step is one pass of the whole path over one batch of synthetic input:
-  1. bsattn_build_index   causal 256 x 256 block mask -> CSR   (3 small launches)
+  1. bsattn_build_index   causal 256 x 256 block mask -> CSR and the
+                          longest-first row order             (4 small launches)
   2. bsattn_fwd_prefill   BLASST prefill, B1 Hq32/Hkv8 N32768 d128, causal,
                           tiles 128, lambda = a / N                (1 launch)
   3. bsattn_fwd_decode    BLASST split-KV decode, B64 Hq32/Hkv8 L131072 d128,
@@ -129,6 +130,7 @@ class Step:
         self.row_ptr = torch.empty(nb + 1, dtype=torch.int32, device="cuda")
         self.col_idx = torch.empty(nb * nb, dtype=torch.int32, device="cuda")
         self.nnz = torch.empty(1, dtype=torch.int32, device="cuda")
+        self.row_order = torch.empty(nb, dtype=torch.int32, device="cuda")
         self.o = torch.empty_like(pw.q)
         self.lse = torch.empty(pw.B, pw.Hq, pw.N, dtype=torch.float32, device="cuda")
         self.do = torch.empty_like(dw.q)
@@ -149,14 +151,16 @@ class Step:
         rc = lib.bsattn_build_index(self.ops._ptr(self.mask), 1, self.pw.nq, self.pw.nk, BLK, BLK, 1,
                                     self.ops._ptr(self.row_ptr), self.ops._ptr(self.col_idx),
                                     self.col_idx.numel(), self.ops._ptr(self.nnz),
-                                    self.ops._ptr(self.status), self.ops._stream(None))
+                                    self.ops._ptr(self.row_order), self.ops._ptr(self.status),
+                                    self.ops._stream(None))
         assert rc == 0
 
     def prefill(self, tile_status=None):
         pw = self.pw
         self.ops.bsattn_fwd_prefill(pw.q, pw.k, pw.v, BLK, pw.scale, True, self.p_lam,
                                     self.row_ptr, self.col_idx, 1, o=self.o, lse=self.lse,
-                                    tile_status=tile_status, status=self.status)
+                                    tile_status=tile_status, status=self.status,
+                                    row_order=self.row_order)
 
     def decode(self, tile_status=None):
         dw = self.dw
@@ -164,7 +168,7 @@ class Step:
                                    o=self.do, lse=self.dlse, workspace=self.ws,
                                    tile_status=tile_status, status=self.status)
 
-    LAUNCHES = 3 + 1 + 2
+    LAUNCHES = 4 + 1 + 2
 
     def counts(self):
         """Visited / executed tiles of this input (decisions are deterministic)."""

@@ -138,7 +138,7 @@ int bsattn_debug_trace(int n, int32_t** host_view) {
 int bsattn_build_index(const uint8_t* d_mask, int mask_heads, int nq_blocks, int nk_blocks,
                        int q_block, int k_block, int causal, int32_t* d_row_ptr,
                        int32_t* d_col_idx, int64_t col_capacity, int32_t* d_nnz,
-                       int32_t* d_status, cudaStream_t stream) {
+                       int32_t* d_row_order, int32_t* d_status, cudaStream_t stream) {
   if (!d_mask || !d_row_ptr || !d_nnz || (!d_col_idx && col_capacity > 0))
     return BSATTN_ERR_INVALID_ARG;
   if (mask_heads < 1 || nq_blocks < 1 || nk_blocks < 1 || q_block < 1 || k_block < 1 ||
@@ -148,16 +148,17 @@ int bsattn_build_index(const uint8_t* d_mask, int mask_heads, int nq_blocks, int
     return BSATTN_ERR_UNSUPPORTED;
   if (int rc = check_device()) return rc;
   IndexArgs a{d_mask, mask_heads, nq_blocks, nk_blocks, q_block, k_block, causal ? 1 : 0,
-              d_row_ptr, d_col_idx, col_capacity, d_nnz, d_status};
+              d_row_ptr, d_col_idx, col_capacity, d_nnz, d_row_order, d_status};
   return launch_build_index(a, stream) == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
 
 int bsattn_fwd_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                        int Hq, int Hkv, int N, int d, int block, float scale, int causal,
                        float lambda, const int32_t* row_ptr, const int32_t* col_idx,
-                       int mask_heads, uint8_t* tile_status, int32_t* d_status,
-                       cudaStream_t stream) {
+                       const int32_t* row_order, int mask_heads, uint8_t* tile_status,
+                       int32_t* d_status, cudaStream_t stream) {
   if (!q || !k || !v || !o) return BSATTN_ERR_INVALID_ARG;
+  if (row_order && !row_ptr) return BSATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0) return BSATTN_ERR_INVALID_ARG;
   if (bad_lambda(lambda) || !std::isfinite(scale) || !(scale > 0.f)) return BSATTN_ERR_INVALID_ARG;
   if (row_ptr && (!col_idx || (mask_heads != 1 && mask_heads != Hq))) return BSATTN_ERR_INVALID_ARG;
@@ -183,6 +184,8 @@ int bsattn_fwd_prefill(const void* q, const void* k, const void* v, void* o, flo
   PrefillParams p{};
   p.row_ptr = row_ptr;
   p.col_idx = col_idx;
+  p.row_order = row_order;
+  p.q = static_cast<const __nv_bfloat16*>(q);
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.tile_status = tile_status;
@@ -204,6 +207,14 @@ int bsattn_fwd_prefill(const void* q, const void* k, const void* v, void* o, flo
   p.trace_n = g_trace_n;
 
   cudaError_t e;
+  // Two query heads of one KV head share a CTA and its K/V stream when the
+  // group size is even and both heads walk the same visit list.
+  const bool pair = block == 128 && (Hq / Hkv) % 2 == 0 && (!row_ptr || mask_heads == 1);
+  if (pair) {
+    e = d == 128 ? launch_prefill_pair<128>(tq, tk, tv, p, (int)(items / 2), stream)
+                 : launch_prefill_pair<64>(tq, tk, tv, p, (int)(items / 2), stream);
+    return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+  }
   if (d == 128 && block == 128) e = launch_prefill<128, 128>(tq, tk, tv, p, (int)items, stream);
   else if (d == 64 && block == 128) e = launch_prefill<64, 128>(tq, tk, tv, p, (int)items, stream);
   else if (d == 128 && block == 64) e = launch_prefill<128, 64>(tq, tk, tv, p, (int)items, stream);

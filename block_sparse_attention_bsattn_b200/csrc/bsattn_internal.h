@@ -15,12 +15,15 @@ struct IndexArgs {
   int32_t* col_idx;
   int64_t capacity;
   int32_t* nnz;
+  int32_t* row_order;  // optional: rows of each mask head, longest first
   int32_t* status;
 };
 
 struct PrefillParams {
   const int32_t* row_ptr;
   const int32_t* col_idx;
+  const int32_t* row_order;  // optional: work order of query tiles within a head
+  const __nv_bfloat16* q;
   __nv_bfloat16* o;
   float* lse;
   uint8_t* tile_status;
@@ -65,6 +68,11 @@ cudaError_t launch_build_index(const IndexArgs& a, cudaStream_t stream);
 template <int D, int BLK>
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const PrefillParams& p, int grid, cudaStream_t stream);
+
+template <int D>
+cudaError_t launch_prefill_pair(const CUtensorMap& tq, const CUtensorMap& tk,
+                                const CUtensorMap& tv, const PrefillParams& p, int grid,
+                                cudaStream_t stream);
 
 template <int D, int BLK, int G>
 cudaError_t launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv,

@@ -2,7 +2,8 @@
 // the 0/1 block mask kept as an index of its non-zero blocks; section 3.3:
 // the attention tiling loop walks that index instead of testing every block).
 //
-// Three small launches on the caller's stream:
+// Three small launches on the caller's stream (a fourth for the optional
+// longest-first row order):
 //   count: one warp per (mask head, query block) row counts the kept key
 //          blocks (ballot over 32 columns at a time) into row_ptr[.. + i + 1];
 //   scan:  one CTA turns the counts into absolute offsets (inclusive scan over
@@ -104,6 +105,24 @@ __global__ void index_fill_kernel(IndexArgs a) {
   }
 }
 
+// Longest-first order of the rows of each mask head (one CTA per head): the
+// rank of row i is the number of rows that are longer, plus the number of
+// equally long rows before it, so ties keep ascending row order.  Quadratic in
+// the number of rows, which is small (one per 64 or 128 tokens).
+__global__ void __launch_bounds__(1024) index_order_kernel(IndexArgs a) {
+  const int h = blockIdx.x;
+  const int32_t* rp = a.row_ptr + (int64_t)h * (a.nq + 1);
+  for (int i = threadIdx.x; i < a.nq; i += blockDim.x) {
+    const int32_t li = rp[i + 1] - rp[i];
+    int rank = 0;
+    for (int j = 0; j < a.nq; ++j) {
+      const int32_t lj = rp[j + 1] - rp[j];
+      rank += (lj > li) || (lj == li && j < i);
+    }
+    a.row_order[(int64_t)h * a.nq + rank] = i;
+  }
+}
+
 cudaError_t launch_build_index(const IndexArgs& a, cudaStream_t stream) {
   const int64_t rows = (int64_t)a.mask_heads * a.nq;
   if (rows == 0) return cudaSuccess;
@@ -112,6 +131,7 @@ cudaError_t launch_build_index(const IndexArgs& a, cudaStream_t stream) {
   index_count_kernel<<<grid, threads, 0, stream>>>(a);
   index_scan_kernel<<<1, 1024, 0, stream>>>(a);
   index_fill_kernel<<<grid, threads, 0, stream>>>(a);
+  if (a.row_order) index_order_kernel<<<a.mask_heads, 1024, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,457 @@
+// Block-sparse prefill for two query heads that share a KV head (GQA group of
+// even size): one CTA runs the same query tile of both heads against one K/V
+// stream, so every K and V tile crosses L2 once for two query tiles.
+//
+// Same method as prefill_sm100.cu ("BLASST: Dynamic Blocked Attention Sparsity
+// via Softmax Thresholding", Algorithm 1 and section 4.1; "块稀疏Attention实战"
+// section 3.3): per query tile, visited key tiles in ascending order, S = Q K^T
+// for each, the row max, the skip test against the running max, and for kept
+// tiles P = exp(S - m), the row sums and O += P V.  The two heads' skip
+// decisions are independent.
+//
+// 10 warps:
+//   warp 0      TMA producer: Q of both heads, then K_j (3-stage ring) and V_j
+//               (2-stage ring)
+//   warp 1      TMEM owner, MMA issuer.  The two query tiles ping-pong: after
+//               head A's P is ready its BMM2 and its next BMM1 are issued, then
+//               head B's, so the tensor core works on one head while the other
+//               head's softmax runs.
+//   warps 2..5  softmax of head A, warps 6..9 softmax of head B: one thread per
+//               query row (TMEM lane), vote across the four warps of the head.
+// TMEM: S_A [0,128)  O_A [128,256)  S_B [256,384)  O_B [384,512).
+// BMM1: A = Q (smem, K-major, 128B swizzle), B = K tile (smem, K-major).
+// BMM2: A = P (TMEM, bf16 over S), B = V tile (smem, MN-major).
+#include <cmath>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "bsattn_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace bsattn {
+
+template <int D>
+struct PairCfg {
+  static constexpr int BLK = 128;
+  static constexpr int KST = 3;
+  static constexpr int VST = 2;
+  static constexpr int HALVES = D / 64;
+  static constexpr int Q_HALF = 128 * 128;
+  static constexpr int T_HALF = BLK * 128;
+  static constexpr int Q_BYTES = HALVES * Q_HALF;
+  static constexpr int T_BYTES = HALVES * T_HALF;
+  static constexpr int Q_OFF = 0;                       // two heads
+  static constexpr int K_OFF = Q_OFF + 2 * Q_BYTES;
+  static constexpr int V_OFF = K_OFF + KST * T_BYTES;
+  static constexpr int BAR_OFF = V_OFF + VST * T_BYTES;
+  static constexpr int SMEM = BAR_OFF + 512 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int THREADS = 320;
+  static constexpr float TAU = 8.0f;
+};
+
+struct PairBarriers {
+  uint64_t q_full;
+  uint64_t k_full[3], k_empty[3];
+  uint64_t v_full[2], v_empty[2];
+  uint64_t s_full[2];       // per head
+  uint64_t p_ready[2];      // per head
+  uint64_t o_done[2];       // per head
+  uint64_t vote_bar[2][2];  // per head, tile parity
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int skip_flag[2];
+  int vote[2][2][4];        // head, tile parity, warp
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
+                        const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+  using C = PairCfg<D>;
+  constexpr int BLK = C::BLK;
+  static_assert(sizeof(PairBarriers) <= 512, "barrier block");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* q_smem = smem + C::Q_OFF;
+  uint8_t* k_smem = smem + C::K_OFF;
+  uint8_t* v_smem = smem + C::V_OFF;
+  PairBarriers* bars = reinterpret_cast<PairBarriers*>(smem + C::BAR_OFF);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  // ---- work item: (batch, head pair, query tile); heads 2*pr and 2*pr + 1
+  // share KV head (2*pr) / group
+  const int PH = p.Hq / 2;
+  const int BP = p.B * PH;
+  int i, bp;
+  if (p.row_order) {
+    bp = (int)(blockIdx.x / p.nq);
+    i = p.row_order[(int)(blockIdx.x % p.nq)];
+  } else if (p.causal) {
+    i = p.nq - 1 - (int)(blockIdx.x / BP);
+    bp = (int)(blockIdx.x % BP);
+  } else {
+    bp = (int)(blockIdx.x / p.nq);
+    i = (int)(blockIdx.x % p.nq);
+  }
+  const int b = bp / PH, h0 = 2 * (bp % PH);
+  const int kvh = h0 / (p.Hq / p.Hkv);
+
+  // ---- visit list (mask head 0: both heads share it)
+  const int32_t* cols = nullptr;
+  int n;
+  if (p.row_ptr) {
+    const int32_t s0 = p.row_ptr[i];
+    const int32_t s1 = p.row_ptr[i + 1];
+    cols = p.col_idx + s0;
+    n = s1 - s0;
+    if (p.causal)
+      while (n > 0 && cols[n - 1] > i) --n;
+  } else {
+    n = p.causal ? i + 1 : p.nk;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < C::KST; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->p_ready[s], 4);
+      mbar_init(&bars->o_done[s], 1);
+      mbar_init(&bars->vote_bar[s][0], 4);
+      mbar_init(&bars->vote_bar[s][1], 4);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const uint64_t lim = p.wait_limit_ns;
+
+  if (warp == 0) {
+    // ======================================================== TMA producer
+    if (lane == 0 && n > 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      if (!p.debug_stall) {
+        mbar_arrive_expect_tx(&bars->q_full, 2 * C::HALVES * BLK * 128);
+        for (int e = 0; e < 2; ++e)
+          for (int hf = 0; hf < C::HALVES; ++hf)
+            tma_load_3d(q_smem + e * C::Q_BYTES + hf * C::Q_HALF, &tmQ, &bars->q_full, hf * 64,
+                        i * BLK, b * p.Hq + h0 + e);
+      }
+      int issued_k = 0, issued_v = 0;
+      for (int t = 0; t < n; ++t) {
+        const int j = cols ? cols[t] : t;
+        const int ks = t % C::KST;
+        if (!mbar_wait(&bars->k_empty[ks], ((t / C::KST) & 1) ^ 1, abort, lim)) break;
+        mbar_arrive_expect_tx(&bars->k_full[ks], C::T_BYTES);
+        for (int hf = 0; hf < C::HALVES; ++hf)
+          tma_load_3d(k_smem + ks * C::T_BYTES + hf * C::T_HALF, &tmK, &bars->k_full[ks],
+                      hf * 64, j * BLK, b * p.Hkv + kvh);
+        ++issued_k;
+        const int vs = t % C::VST;
+        if (!mbar_wait(&bars->v_empty[vs], ((t / C::VST) & 1) ^ 1, abort, lim)) break;
+        mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
+        for (int hf = 0; hf < C::HALVES; ++hf)
+          tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
+                      hf * 64, j * BLK, b * p.Hkv + kvh);
+        ++issued_v;
+      }
+      if (*abort) {
+        for (int t = (issued_k > C::KST ? issued_k - C::KST : 0); t < issued_k; ++t)
+          mbar_wait_drain(&bars->k_full[t % C::KST], (t / C::KST) & 1, lim);
+        for (int t = (issued_v > C::VST ? issued_v - C::VST : 0); t < issued_v; ++t)
+          mbar_wait_drain(&bars->v_full[t % C::VST], (t / C::VST) & 1, lim);
+        if (!p.debug_stall) mbar_wait_drain(&bars->q_full, 0, lim);
+      }
+    }
+  } else if (warp == 1) {
+    // ======================================================== MMA issuer
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t IDESC1 = idesc_bf16_f32(128, BLK, 0, 0);
+      constexpr uint32_t IDESC2 = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_addr = smem_u32(q_smem);
+      const uint32_t k_addr = smem_u32(k_smem);
+      const uint32_t v_addr = smem_u32(v_smem);
+      bool ok = mbar_wait(&bars->q_full, 0, abort, lim);
+      tc_fence_after();
+      // S_e = Q_e K_t^T into TMEM columns [256 e, 256 e + 128)
+      auto bmm1 = [&](int e, int t) {
+        const int ks = t % C::KST;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t a = q_addr + e * C::Q_BYTES + (kk / 4) * C::Q_HALF + (kk % 4) * 32;
+          const uint32_t bb = k_addr + ks * C::T_BYTES + (kk / 4) * C::T_HALF + (kk % 4) * 32;
+          mma_ss(tmem + 256 * e, smem_desc(a, 16, 1024, 2), smem_desc(bb, 16, 1024, 2), IDESC1,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->s_full[e]);
+      };
+      // O_e += P_e V_t, P_e in TMEM over S_e
+      auto bmm2 = [&](int e, int t, int first) {
+        const int vs = t % C::VST;
+#pragma unroll
+        for (int kk = 0; kk < BLK / 16; ++kk) {
+          const uint32_t bb = v_addr + vs * C::T_BYTES + kk * (16 * 128);
+          mma_ts(tmem + 256 * e + 128, tmem + 256 * e + kk * 8, smem_desc(bb, C::T_HALF, 1024, 2),
+                 IDESC2, (!first || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&bars->o_done[e]);
+      };
+      if (ok) {
+        ok = mbar_wait(&bars->k_full[0], 0, abort, lim);
+        tc_fence_after();
+        if (ok) {
+          bmm1(0, 0);
+          bmm1(1, 0);
+          mma_commit(&bars->k_empty[0]);
+        }
+      }
+      int kept[2] = {0, 0};
+      for (int t = 0; ok && t < n; ++t) {
+        const int vs = t % C::VST;
+        bool v_ready = false;
+        const bool more = t + 1 < n;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          if (!mbar_wait(&bars->p_ready[e], t & 1, abort, lim)) { ok = false; break; }
+          tc_fence_after();
+          const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[e]);
+          if (!skip) {
+            if (!v_ready) {
+              if (!mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) { ok = false; break; }
+              tc_fence_after();
+              v_ready = true;
+            }
+            bmm2(e, t, kept[e] == 0);
+            ++kept[e];
+          }
+          if (more) {
+            if (e == 0) {   // first use of K_{t+1}
+              const int ks = (t + 1) % C::KST;
+              if (!mbar_wait(&bars->k_full[ks], ((t + 1) / C::KST) & 1, abort, lim)) { ok = false; break; }
+              tc_fence_after();
+            }
+            bmm1(e, t + 1);
+          }
+        }
+        if (!ok) break;
+        if (more) mma_commit(&bars->k_empty[(t + 1) % C::KST]);
+        // release V_t: consumed (or not needed) by both heads
+        if (!v_ready) {
+          if (!mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) break;
+          mbar_arrive(&bars->v_empty[vs]);
+        } else {
+          mma_commit(&bars->v_empty[vs]);
+        }
+      }
+      mma_commit(&bars->drain);
+      mbar_wait_drain(&bars->drain, 0, lim);
+    }
+  } else {
+    // ======================================================== softmax warps
+    const int e = (warp - 2) / 4;           // which head of the pair
+    const int sw = (warp - 2) % 4;
+    const int quarter = warp % 4;
+    const int row = quarter * 32 + lane;
+    const int r0 = i * BLK;
+    const int h = h0 + e;
+    const bool valid = r0 + row < p.N;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t s_col = 256 * e, o_col = 256 * e + 128;
+    float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
+    int kept = 0;
+    bool ok = true;
+    for (int t = 0; t < n; ++t) {
+      const int j = cols ? cols[t] : t;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[e], t & 1, abort, lim))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[BLK];
+#pragma unroll
+      for (int c0 = 0; c0 < BLK; c0 += 32)
+        tmem_ld32(lane_addr + s_col + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
+      tmem_wait_ld();
+      const int k0 = j * BLK;
+      if (k0 + BLK > p.N || (p.causal && j == i)) {
+        const int qpos = r0 + row;
+#pragma unroll
+        for (int c = 0; c < BLK; ++c) {
+          const int key = k0 + c;
+          if (key >= p.N || (p.causal && key > qpos)) r[c] = __float_as_uint(-INFINITY);
+        }
+      }
+      float m8[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) m8[x] = __uint_as_float(r[x]);
+#pragma unroll
+      for (int c = 8; c < BLK; c += 8)
+#pragma unroll
+        for (int x = 0; x < 8; ++x) m8[x] = fmaxf(m8[x], __uint_as_float(r[c + x]));
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      const float mt = mx * p.scale_log2;
+      int skip = 0;
+      if (p.use_skip) {
+        const bool pass = !valid || (mt - m_run < p.thr_log2);
+        const bool wpass = __all_sync(0xffffffffu, pass);
+        if (lane == 0) {
+          bars->vote[e][t & 1][sw] = wpass ? 1 : 0;
+          mbar_arrive(&bars->vote_bar[e][t & 1]);
+        }
+        __syncwarp();
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&bars->vote_bar[e][t & 1], (t >> 1) & 1, abort, lim))) {
+          ok = false;
+          break;
+        }
+        volatile int* vv = bars->vote[e][t & 1];
+        skip = vv[0] & vv[1] & vv[2] & vv[3];
+      }
+      m_run = fmaxf(m_run, mt);
+      if (sw == 0 && lane == 0 && p.tile_status && (unsigned)j < (unsigned)p.nk)
+        p.tile_status[(((int64_t)b * p.Hq + h) * p.nq + i) * p.nk + j] = skip ? 1 : 2;
+      if (!skip) {
+        if (kept > 0) {
+          // S_e holds this tile, so BMM2 of the previous kept tile has finished
+          // reading P; wait for it to land in O before O may be rescaled
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[e], (kept - 1) & 1, abort, lim))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        float alpha = 1.f;
+        bool rescale = false;
+        if (kept == 0) {
+          m_ref = m_run;
+        } else if (m_run > m_ref + C::TAU) {
+          alpha = fast_exp2(m_ref - m_run);
+          rescale = true;
+          m_ref = m_run;
+        }
+        const float shift = (m_ref == -INFINITY) ? 0.f : m_ref;
+        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c0 = 0; c0 < BLK; c0 += 32) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(r[c0 + c]), p.scale_log2, -shift));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(r[c0 + c + 1]), p.scale_log2, -shift));
+            rs8[(c / 2) & 7] += p0 + p1;
+            pk[c / 2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(lane_addr + s_col + c0 / 2, pk);
+        }
+        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) +
+                         ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        l = l * alpha + rs;
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ro[32];
+            tmem_ld32(lane_addr + o_col + c0, ro);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ro[c] = __float_as_uint(__uint_as_float(ro[c]) * alpha);
+            tmem_st32(lane_addr + o_col + c0, ro);
+          }
+        }
+        tmem_wait_st();
+        ++kept;
+      }
+      if (sw == 0 && lane == 0) bars->skip_flag[e] = skip;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_ready[e]);
+    }
+    // ---- epilogue
+    if (ok && kept > 0) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[e], (kept - 1) & 1, abort, lim)))
+        ok = false;
+      tc_fence_after();
+    }
+    if (ok) {
+      const int64_t orow = ((int64_t)b * p.Hq + h) * p.N + r0 + row;
+      __nv_bfloat16* dst = p.o + orow * D;
+      const bool have = kept > 0 && l > 0.f;
+      const float inv_l = have ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t ro[32];
+        if (kept > 0) {
+          tmem_ld32(lane_addr + o_col + c0, ro);
+          tmem_wait_ld();
+        }
+        if (valid) {
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float a0 = have ? __uint_as_float(ro[c]) * inv_l : 0.f;
+            const float a1 = have ? __uint_as_float(ro[c + 1]) * inv_l : 0.f;
+            w[c / 2] = pack_bf16x2(a0, a1);
+          }
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        }
+      }
+      if (valid && p.lse)
+        p.lse[orow] = have ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && bars->abort) report_status(p.status, kDevTimeout);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+cudaError_t launch_prefill_pair(const CUtensorMap& tq, const CUtensorMap& tk,
+                                const CUtensorMap& tv, const PrefillParams& p, int grid,
+                                cudaStream_t stream) {
+  using C = PairCfg<D>;
+  static_assert(C::SMEM <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(prefill_pair_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  prefill_pair_kernel<D><<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_prefill_pair<128>(const CUtensorMap&, const CUtensorMap&,
+                                              const CUtensorMap&, const PrefillParams&, int,
+                                              cudaStream_t);
+template cudaError_t launch_prefill_pair<64>(const CUtensorMap&, const CUtensorMap&,
+                                             const CUtensorMap&, const PrefillParams&, int,
+                                             cudaStream_t);
+
+}  // namespace bsattn

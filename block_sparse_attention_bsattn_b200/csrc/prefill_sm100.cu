@@ -10,20 +10,21 @@
 // (CUDA cores), the row sums, and O += P V (BMM2).  A skipped tile costs one
 // BMM1 and a row max.
 //
-// One CTA = one (batch, head, query tile) work item; 6 warps:
+// One CTA = one (batch, head, query tile) work item; 10 warps:
 //   warp 0      TMA producer: Q once, then K_j and V_j of every visited tile
-//               into 2-stage rings (V is loaded for every visited tile, as the
+//               into 3-stage rings (V is loaded for every visited tile, as the
 //               BLASST prefill kernel does -- the load is not on the critical
 //               path of a compute-bound kernel);
 //   warp 1      TMEM owner and MMA issuer (one elected lane): BMM1 of tile
 //               t + 1 is issued before waiting for the softmax of tile t, so
 //               the tensor core works while the softmax warps do;
-//   warps 2..5  softmax: one thread per query row (TMEM lane), skip vote
-//               (__all_sync per warp, then one shared-memory flag and one
-//               mbarrier arrival per warp to agree across the four warps),
-//               P = exp2 written back to
-//               TMEM as bf16 over the tile's S columns, lazy rescale of O, and
-//               the epilogue.
+//   warps 2..9  softmax, two warpgroups: each query row (TMEM lane) is shared
+//               by one thread of each warpgroup, which own the low and the
+//               high half of the score columns (and of the output columns).
+//               Per tile one shared-memory round exchanges the half-row maxima
+//               and the warp votes (__all_sync per warp; a row passes iff both
+//               halves pass); P = exp2 goes back to TMEM as bf16 over the
+//               tile's S columns; lazy rescale of O; the epilogue.
 // TMEM columns: S double buffer at [0,128) and [128,256), O at [256, 256+d).
 // BMM1: A = Q (smem, K-major, 128B swizzle), B = K tile (smem, K-major).
 // BMM2: A = P (TMEM), B = V tile (smem, MN-major, 128B swizzle).
@@ -42,17 +43,15 @@ namespace bsattn {
 
 template <int D, int BLK>
 struct PrefillCfg {
-  static constexpr int KST = 2;                    // K ring stages
-  static constexpr int VST = 2;                    // V ring stages
+  static constexpr int KST = 3;                    // K ring stages
+  static constexpr int VST = 3;                    // V ring stages
   static constexpr int HALVES = D / 64;            // 64-column (128-byte) swizzle boxes
-  static constexpr int Q_HALF = 128 * 128;         // bytes per Q box region (128 rows)
   static constexpr int T_HALF = BLK * 128;         // bytes per K/V box region
-  static constexpr int Q_BYTES = HALVES * Q_HALF;
   static constexpr int T_BYTES = HALVES * T_HALF;
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + Q_BYTES;
+  static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + KST * T_BYTES;
-  static constexpr int BAR_OFF = V_OFF + VST * T_BYTES;
+  static constexpr int XM_OFF = V_OFF + VST * T_BYTES;  // float [2][2][128] + [2][128]
+  static constexpr int BAR_OFF = XM_OFF + 6 * 128 * 4;
   // + alignment slack; at least 116 KB so that one CTA (which holds all 512
   // TMEM columns) is resident per SM
   static constexpr int SMEM_USED = BAR_OFF + 256 + 1024;
@@ -60,27 +59,29 @@ struct PrefillCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0;             // S[b] at b * 128
   static constexpr uint32_t O_COL = 256;
-  static constexpr int THREADS = 192;
+  static constexpr uint32_t Q_COL = 384;           // Q tile, bf16 pairs (d/2 columns)
+  static constexpr int THREADS = 320;
   static constexpr float TAU = 8.0f;               // lazy-rescale slack (base-2 units)
 };
 
 struct PrefillBarriers {
-  uint64_t q_full;
-  uint64_t k_full[2], k_empty[2];
-  uint64_t v_full[2], v_empty[2];
+  uint64_t q_ready;      // Q written to TMEM by the softmax warps
+  uint64_t k_full[3], k_empty[3];
+  uint64_t v_full[3], v_empty[3];
   uint64_t s_full[2];
   uint64_t p_ready[2];
   uint64_t o_done;
   uint64_t drain;
   uint64_t vote_bar[2];
+  uint64_t epi_bar;
   uint32_t tmem_base;
   int abort;
   int skip_flag[2];
-  int vote[2][4];
+  int vote[2][8];
 };
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   using C = PrefillCfg<D, BLK>;
@@ -88,7 +89,6 @@ __global__ void __launch_bounds__(192, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* q_smem = smem + C::Q_OFF;
   uint8_t* k_smem = smem + C::K_OFF;
   uint8_t* v_smem = smem + C::V_OFF;
   PrefillBarriers* bars = reinterpret_cast<PrefillBarriers*>(smem + C::BAR_OFF);
@@ -96,10 +96,17 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // ---- work item (longest-first for causal: query tiles in descending order)
+  // ---- work item.  With a row order (longest rows first, from the index
+  // builder) the items of one head run together, longest first; otherwise
+  // causal work runs in descending query-tile order (longest first) and
+  // non-causal work head by head.
   const int BH = p.B * p.Hq;
   int i, bh;
-  if (p.causal) {
+  if (p.row_order) {
+    bh = (int)(blockIdx.x / p.nq);
+    const int mh_o = p.mask_heads == 1 ? 0 : bh % p.Hq;
+    i = p.row_order[(int64_t)mh_o * p.nq + (int)(blockIdx.x % p.nq)];
+  } else if (p.causal) {
     i = p.nq - 1 - (int)(blockIdx.x / BH);
     bh = (int)(blockIdx.x % BH);
   } else {
@@ -124,24 +131,37 @@ __global__ void __launch_bounds__(192, 1)
     n = p.causal ? i + 1 : p.nk;
   }
 
-  // debug trace: slot 16 + CTA = stage reached; CTA 0 also records per-role progress
+  // debug trace: slot 16 + CTA = stage reached; CTA 0 also records per-role
+  // progress, and an SM-clock timeline of its first tiles from slot 1024 on
+  // (8 slots per tile: BMM1 issued, P seen by the MMA warp, BMM2 issued, S seen
+  // by the softmax, votes agreed, P handed back)
   const bool tr0 = blockIdx.x == 0;
+  auto tl_mark = [&](int t, int k) {   // plain store: no fence, read after the kernel
+    if (tr0 && p.trace && 1024 + t * 8 + k < p.trace_n) {
+      p.trace[1024 + t * 8 + k] = (int32_t)clock64();
+    }
+  };
   if (threadIdx.x == 0) trace_mark(p.trace, p.trace_n, 16 + blockIdx.x, 1);
 
   // ---- setup
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    mbar_init(&bars->q_ready, 8);
+    for (int s = 0; s < C::KST; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < C::VST; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_ready[s], 4);
+      mbar_init(&bars->p_ready[s], 8);
     }
     mbar_init(&bars->o_done, 1);
-    mbar_init(&bars->vote_bar[0], 4);
-    mbar_init(&bars->vote_bar[1], 4);
+    mbar_init(&bars->vote_bar[0], 8);
+    mbar_init(&bars->vote_bar[1], 8);
+    mbar_init(&bars->epi_bar, 8);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_barrier_init();
@@ -160,15 +180,8 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     // ======================================================== TMA producer
     if (lane == 0 && n > 0) {
-      prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      if (!p.debug_stall) {
-        mbar_arrive_expect_tx(&bars->q_full, C::HALVES * BLK * 128);
-        for (int hf = 0; hf < C::HALVES; ++hf)
-          tma_load_3d(q_smem + hf * C::Q_HALF, &tmQ, &bars->q_full, hf * 64, i * BLK,
-                      b * p.Hq + h);
-      }
       int issued_k = 0, issued_v = 0;
       for (int t = 0; t < n; ++t) {
         const int j = cols ? cols[t] : t;
@@ -195,8 +208,6 @@ __global__ void __launch_bounds__(192, 1)
           mbar_wait_drain(&bars->k_full[t % C::KST], (t / C::KST) & 1, lim);
         for (int t = (issued_v > C::VST ? issued_v - C::VST : 0); t < issued_v; ++t)
           mbar_wait_drain(&bars->v_full[t % C::VST], (t / C::VST) & 1, lim);
-        if (!p.debug_stall)
-          mbar_wait_drain(&bars->q_full, 0, lim);
       }
     }
   } else if (warp == 1) {
@@ -204,10 +215,9 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0 && n > 0) {
       constexpr uint32_t IDESC1 = idesc_bf16_f32(128, BLK, 0, 0);
       constexpr uint32_t IDESC2 = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_addr = smem_u32(q_smem);
       const uint32_t k_addr = smem_u32(k_smem);
       const uint32_t v_addr = smem_u32(v_smem);
-      bool ok = mbar_wait(&bars->q_full, 0, abort, lim);
+      bool ok = mbar_wait(&bars->q_ready, 0, abort, lim);
       tc_fence_after();
       auto issue_bmm1 = [&](int t) -> bool {
         const int ks = t % C::KST;
@@ -216,13 +226,13 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t d_tmem = tmem + C::S_COL + (uint32_t)(t & 1) * 128u;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a = q_addr + (kk / 4) * C::Q_HALF + (kk % 4) * 32;
           const uint32_t bb = k_addr + ks * C::T_BYTES + (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(d_tmem, smem_desc(a, 16, 1024, 2), smem_desc(bb, 16, 1024, 2), IDESC1,
+          mma_ts(d_tmem, tmem + C::Q_COL + kk * 8, smem_desc(bb, 16, 1024, 2), IDESC1,
                  kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars->s_full[t & 1]);
         mma_commit(&bars->k_empty[ks]);
+        tl_mark(t, 0);
         return true;
       };
       if (ok) ok = issue_bmm1(0);
@@ -232,6 +242,7 @@ __global__ void __launch_bounds__(192, 1)
         const int sb = t & 1;
         if (!mbar_wait(&bars->p_ready[sb], (t >> 1) & 1, abort, lim)) break;
         tc_fence_after();
+        tl_mark(t, 1);
         const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[sb]);
         const int vs = t % C::VST;
         if (!mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) break;
@@ -246,6 +257,7 @@ __global__ void __launch_bounds__(192, 1)
           }
           mma_commit(&bars->o_done);
           mma_commit(&bars->v_empty[vs]);
+          tl_mark(t, 2);
           ++kept;
         } else {
           mbar_arrive(&bars->v_empty[vs]);
@@ -260,16 +272,46 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ======================================================== softmax warps
+    // Two warpgroups share every query row: warpgroup `half` owns the score
+    // columns [half*CW, half*CW + CW) and the output columns
+    // [half*OW, half*OW + OW) of the rows of its TMEM lane quarter.
+    constexpr int CW = BLK / 2;
+    constexpr int OW = D / 2;
+    const int sw = warp - 2;                // 0..7
+    const int half = sw / 4;
     const int quarter = warp % 4;           // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;    // query row inside the tile
     const int r0 = i * BLK;
     const bool in_tile = row < BLK;
     const bool valid = in_tile && (r0 + row < p.N);
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int sw = warp - 2;                // 0..3
-    float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
+    float* xmax = reinterpret_cast<float*>(smem + C::XM_OFF);   // [2][2][128]
+    float* lx = xmax + 2 * 2 * 128;                               // [2][128]
+    float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;          // l: this half's columns
     int kept = 0;
     bool ok = true;
+    // Q row -> TMEM (the A operand of BMM1, bf16 pairs along d): warpgroup
+    // `half` writes d in [half*OW, half*OW + OW); rows past N are zero
+    if (n > 0 && in_tile) {
+      const uint4* qsrc = reinterpret_cast<const uint4*>(
+          p.q + (((int64_t)b * p.Hq + h) * p.N + r0 + row) * D + half * OW);
+#pragma unroll
+      for (int c0 = 0; c0 < OW / 2; c0 += 16) {        // 16 columns = 32 bf16 = 4 x uint4
+        uint32_t w[16];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 x = (r0 + row < p.N) ? qsrc[c0 / 4 + v] : make_uint4(0, 0, 0, 0);
+          w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+        }
+        tmem_st16(lane_addr + C::Q_COL + half * (OW / 2) + c0, w);
+      }
+      tmem_wait_st();
+    }
+    if (n > 0 && !p.debug_stall) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->q_ready);
+    }
     for (int t = 0; t < n; ++t) {
       const int j = cols ? cols[t] : t;
       const int sb = t & 1;
@@ -278,58 +320,65 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       tc_fence_after();
-      float s[BLK];
+      if (sw == 0 && lane == 0) tl_mark(t, 3);
+      float s[CW];
+      float mh = -INFINITY;
       if (in_tile) {
+        uint32_t r[CW];
 #pragma unroll
-        for (int c0 = 0; c0 < BLK; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(lane_addr + C::S_COL + sb * 128 + c0, r);
-          tmem_wait_ld();
+        for (int c0 = 0; c0 < CW; c0 += 32)
+          tmem_ld32(lane_addr + C::S_COL + sb * 128 + half * CW + c0,
+                    *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
+        tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) s[c0 + c] = __uint_as_float(r[c]);
-        }
+        for (int c = 0; c < CW; ++c) s[c] = __uint_as_float(r[c]);
         // element masks: keys past the end, and keys after the query (causal)
-        const int k0 = j * BLK;
-        if (k0 + BLK > p.N || (p.causal && j == i)) {
+        const int k0 = j * BLK + half * CW;
+        if (j * BLK + BLK > p.N || (p.causal && j == i)) {
           const int qpos = r0 + row;
 #pragma unroll
-          for (int c = 0; c < BLK; ++c) {
+          for (int c = 0; c < CW; ++c) {
             const int key = k0 + c;
             if (key >= p.N || (p.causal && key > qpos)) s[c] = -INFINITY;
           }
         }
-      }
-      float mx = -INFINITY;
-      if (in_tile) {
+        float m8[8];
 #pragma unroll
-        for (int c = 0; c < BLK; ++c) mx = fmaxf(mx, s[c]);
+        for (int e = 0; e < 8; ++e) m8[e] = s[e];
+#pragma unroll
+        for (int c = 8; c < CW; c += 8)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], s[c + e]);
+        mh = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       }
-      const float mt = mx * p.scale_log2;  // tile row max, base-2 units
+      const float mth = mh * p.scale_log2;  // half-row max, base-2 units
+      // The row passes iff both of its halves pass: max(a, b) - m < t exactly
+      // when a - m < t and b - m < t.  One exchange round carries the warp
+      // votes and the half-row maxima (needed for the running max).
+      const bool pass = !valid || (mth - m_run < p.thr_log2);
+      const bool wpass = __all_sync(0xffffffffu, pass);
+      xmax[((t & 1) * 2 + half) * 128 + row] = mth;
+      if (lane == 0) bars->vote[t & 1][sw] = wpass ? 1 : 0;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->vote_bar[t & 1]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->vote_bar[t & 1], (t >> 1) & 1, abort, lim))) {
+        ok = false;
+        break;
+      }
+      if (sw == 0 && lane == 0) tl_mark(t, 4);
       int skip = 0;
       if (p.use_skip) {
-        // skip only if every valid row is below the running max + log2(lambda)
-        const bool pass = !valid || (mt - m_run < p.thr_log2);
-        const bool wpass = __all_sync(0xffffffffu, pass);
-        if (lane == 0) {
-          bars->vote[t & 1][sw] = wpass ? 1 : 0;
-          mbar_arrive(&bars->vote_bar[t & 1]);
-        }
-        __syncwarp();
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(&bars->vote_bar[t & 1], (t >> 1) & 1, abort, lim))) {
-          ok = false;
-          break;
-        }
         volatile int* vv = bars->vote[t & 1];
-        skip = vv[0] & vv[1] & vv[2] & vv[3];
+        skip = vv[0] & vv[1] & vv[2] & vv[3] & vv[4] & vv[5] & vv[6] & vv[7];
       }
+      const float mt = fmaxf(mth, xmax[((t & 1) * 2 + (half ^ 1)) * 128 + row]);
       m_run = fmaxf(m_run, mt);
       if (sw == 0 && lane == 0 && p.tile_status && (unsigned)j < (unsigned)p.nk)
         p.tile_status[(((int64_t)b * p.Hq + h) * p.nq + i) * p.nk + j] = skip ? 1 : 2;
       if (!skip) {
         if (kept > 0) {
-          // the previous BMM2 must be complete before P overwrites this S
-          // buffer's neighbour state and before O may be rescaled
+          // the previous BMM2 must be complete before O may be rescaled
           if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (kept - 1) & 1, abort, lim))) {
             ok = false;
             break;
@@ -337,7 +386,8 @@ __global__ void __launch_bounds__(192, 1)
           tc_fence_after();
         }
         // exponent shift: set by the first kept tile, then moved only when the
-        // running max exceeds it by more than TAU (O and l rescaled below)
+        // running max exceeds it by more than TAU (O and l rescaled below);
+        // both halves of a row compute the same shift
         float alpha = 1.f;
         bool rescale = false;
         if (kept == 0) {
@@ -349,30 +399,32 @@ __global__ void __launch_bounds__(192, 1)
         }
         const float shift = (m_ref == -INFINITY) ? 0.f : m_ref;
         if (in_tile) {
-          float rs = 0.f;
+          float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c0 = 0; c0 < BLK; c0 += 32) {
+          for (int c0 = 0; c0 < CW; c0 += 32) {
             uint32_t pk[16];
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
               const float p0 = fast_exp2(fmaf(s[c0 + c], p.scale_log2, -shift));
               const float p1 = fast_exp2(fmaf(s[c0 + c + 1], p.scale_log2, -shift));
-              rs += p0 + p1;
+              rs8[(c / 2) & 7] += p0 + p1;
               pk[c / 2] = pack_bf16x2(p0, p1);
             }
-            tmem_st16(lane_addr + C::S_COL + sb * 128 + c0 / 2, pk);
+            tmem_st16(lane_addr + C::S_COL + sb * 128 + (half * CW + c0) / 2, pk);
           }
+          const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) +
+                           ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
           l = l * alpha + rs;
-          // rare: bring the accumulated O to the new shift (no BMM2 is in flight)
+          // rare: bring this half of the accumulated O to the new shift
           if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t r[32];
-              tmem_ld32(lane_addr + C::O_COL + c0, r);
+            for (int c0 = 0; c0 < OW; c0 += 32) {
+              uint32_t ro[32];
+              tmem_ld32(lane_addr + C::O_COL + half * OW + c0, ro);
               tmem_wait_ld();
 #pragma unroll
-              for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-              tmem_st32(lane_addr + C::O_COL + c0, r);
+              for (int c = 0; c < 32; ++c) ro[c] = __float_as_uint(__uint_as_float(ro[c]) * alpha);
+              tmem_st32(lane_addr + C::O_COL + half * OW + c0, ro);
             }
           }
           tmem_wait_st();
@@ -383,27 +435,35 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready[sb]);
-      if (tr0 && lane == 0) trace_mark(p.trace, p.trace_n, 4 + sw, t + 1);
+      if (sw == 0 && lane == 0) tl_mark(t, 5);
+      if (tr0 && lane == 0) trace_mark(p.trace, p.trace_n, 4 + (sw & 3), t + 1);
     }
 
-    // ---- epilogue: O / l -> bf16, LSE.  tcgen05.ld is warp-collective, so
-    // every lane of a warp that owns tile rows loads; only rows inside the
-    // sequence are stored.
+    // ---- epilogue: row sums of both halves, O / l -> bf16, LSE.  tcgen05.ld
+    // is warp-collective, so every lane of a warp that owns tile rows loads;
+    // only rows inside the sequence are stored.
+    if (ok) {
+      lx[half * 128 + row] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->epi_bar);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->epi_bar, 0, abort, lim))) ok = false;
+    }
     if (ok && kept > 0) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (kept - 1) & 1, abort, lim)))
         ok = false;
       tc_fence_after();
     }
     if (ok && in_tile) {
+      const float lt = lx[row] + lx[128 + row];
       const int64_t orow = ((int64_t)b * p.Hq + h) * p.N + r0 + row;
-      __nv_bfloat16* dst = p.o + orow * D;
-      const bool have = kept > 0 && l > 0.f;
-      const float inv_l = have ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = p.o + orow * D + half * OW;
+      const bool have = kept > 0 && lt > 0.f;
+      const float inv_l = have ? 1.f / lt : 0.f;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < OW; c0 += 32) {
         uint32_t r[32];
         if (kept > 0) {
-          tmem_ld32(lane_addr + C::O_COL + c0, r);
+          tmem_ld32(lane_addr + C::O_COL + half * OW + c0, r);
           tmem_wait_ld();
         }
         if (valid) {
@@ -420,8 +480,8 @@ __global__ void __launch_bounds__(192, 1)
             d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
-      if (valid && p.lse)
-        p.lse[orow] = have ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      if (valid && half == 0 && p.lse)
+        p.lse[orow] = have ? (m_ref + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
     }
   }
 

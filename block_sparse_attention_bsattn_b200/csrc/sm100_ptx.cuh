@@ -250,11 +250,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// Debug progress marker: slot `i` of a host-visible trace buffer (no-op when
-// tracing is off).  Stores are volatile and fenced at system scope so that a
-// host thread can watch them while the kernel runs.
+// Debug progress marker: slot `i` (< 1024) of a host-visible trace buffer
+// (no-op when tracing is off).  Stores are volatile and fenced at system scope
+// so that a host thread can watch them while the kernel runs.
 __device__ __forceinline__ void trace_mark(volatile int32_t* trace, int n, int i, int32_t v) {
-  if (trace && i < n) {
+  if (trace && i < n && i < 1024) {
     trace[i] = v;
     __threadfence_system();
   }

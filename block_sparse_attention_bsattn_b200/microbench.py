@@ -41,6 +41,7 @@ def main():
     ap.add_argument("--a", type=float, default=10.0)
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=2)
+    ap.add_argument("--no-order", action="store_true", help="static masks: no longest-first order")
     args = ap.parse_args()
     torch.cuda.set_device(0)
     out = {"what": args.what}
@@ -63,9 +64,11 @@ def main():
         w = inputs.workload(args.what, device="cuda", generate=False)
         q, k, v = inputs.normal_qkv(1, args.heads, args.heads, w.N, w.d, "cuda", 1236)
         m = w.mask.cuda()
-        rp, ci, nnz = ops.bsattn_build_index(m, w.block, w.block, False)
+        rp, ci, nnz, order = ops.bsattn_build_index(m, w.block, w.block, False, with_order=True)
+        if args.no_order:
+            order = None
         fn = lambda: ops.bsattn_fwd_prefill(q, k, v, w.block, w.scale, False, 0.0, rp, ci, 1,
-                                            want_lse=False)
+                                            want_lse=False, row_order=order)
         for _ in range(args.warmup):
             fn()
         ms = _time(fn, args.iters)

@@ -37,10 +37,10 @@ _lib.bsattn_debug_set.argtypes = [ctypes.c_longlong, _I]
 _lib.bsattn_debug_set.restype = _I
 _lib.bsattn_debug_trace.argtypes = [_I, ctypes.POINTER(ctypes.POINTER(ctypes.c_int32))]
 _lib.bsattn_debug_trace.restype = _I
-_lib.bsattn_build_index.argtypes = [_P, _I, _I, _I, _I, _I, _I, _P, _P, _I64, _P, _P, _P]
+_lib.bsattn_build_index.argtypes = [_P, _I, _I, _I, _I, _I, _I, _P, _P, _I64, _P, _P, _P, _P]
 _lib.bsattn_build_index.restype = _I
 _lib.bsattn_fwd_prefill.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F,
-                                    _P, _P, _I, _P, _P, _P]
+                                    _P, _P, _P, _I, _P, _P, _P]
 _lib.bsattn_fwd_prefill.restype = _I
 _lib.bsattn_decode_workspace_size.argtypes = [_I, _I, _I, _I]
 _lib.bsattn_decode_workspace_size.restype = _SZ
@@ -108,10 +108,11 @@ def _check(t: torch.Tensor, name: str, dtype, dims: int):
 
 def bsattn_build_index(mask: torch.Tensor, q_block: int, k_block: int, causal: bool = False,
                        capacity: Optional[int] = None, status: Optional[torch.Tensor] = None,
-                       stream=None):
+                       with_order: bool = False, stream=None):
     """mask uint8 [mask_heads, nq, nk] -> (row_ptr int32 [mask_heads*(nq+1)],
-    col_idx int32 [capacity], nnz int32 [mask_heads]); col_idx is sized to
-    `capacity` (default: every block)."""
+    col_idx int32 [capacity], nnz int32 [mask_heads]) and, with `with_order`,
+    a fourth tensor row_order int32 [mask_heads*nq] (longest rows first).
+    col_idx is sized to `capacity` (default: every block)."""
     if mask.dim() == 2:
         mask = mask[None]
     _check(mask, "mask", torch.uint8, 3)
@@ -121,11 +122,14 @@ def bsattn_build_index(mask: torch.Tensor, q_block: int, k_block: int, causal: b
     row_ptr = torch.empty(Hm * (nq + 1), dtype=torch.int32, device=dev)
     col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
     nnz = torch.empty(Hm, dtype=torch.int32, device=dev)
+    order = torch.empty(Hm * nq, dtype=torch.int32, device=dev) if with_order else None
     rc = _lib.bsattn_build_index(_ptr(mask), Hm, nq, nk, int(q_block), int(k_block), int(causal),
-                                 _ptr(row_ptr), _ptr(col_idx), cap, _ptr(nnz), _ptr(status),
-                                 _stream(stream))
+                                 _ptr(row_ptr), _ptr(col_idx), cap, _ptr(nnz), _ptr(order),
+                                 _ptr(status), _stream(stream))
     if rc:
         raise BsattnError(rc, "bsattn_build_index")
+    if with_order:
+        return row_ptr, col_idx, nnz, order
     return row_ptr, col_idx, nnz
 
 
@@ -135,7 +139,8 @@ def bsattn_fwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
                        col_idx: Optional[torch.Tensor] = None, mask_heads: int = 1,
                        o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                        want_lse: bool = True, tile_status: Optional[torch.Tensor] = None,
-                       status: Optional[torch.Tensor] = None, stream=None):
+                       status: Optional[torch.Tensor] = None,
+                       row_order: Optional[torch.Tensor] = None, stream=None):
     """q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 -> (o [B,Hq,N,d] bf16, lse [B,Hq,N] fp32 or None)."""
     _check(q, "q", torch.bfloat16, 4)
     _check(k, "k", torch.bfloat16, 4)
@@ -152,8 +157,8 @@ def bsattn_fwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
         lse = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
     rc = _lib.bsattn_fwd_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
                                  int(block), float(scale), int(causal), float(lam), _ptr(row_ptr),
-                                 _ptr(col_idx), int(mask_heads), _ptr(tile_status), _ptr(status),
-                                 _stream(stream))
+                                 _ptr(col_idx), _ptr(row_order), int(mask_heads),
+                                 _ptr(tile_status), _ptr(status), _stream(stream))
     if rc:
         raise BsattnError(rc, "bsattn_fwd_prefill")
     return o, lse

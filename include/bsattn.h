@@ -96,6 +96,10 @@ int bsattn_debug_trace(int n, int32_t **host_view);
  *               d_col_idx (head h's rows follow head h-1's)
  *   d_col_idx   int32 [col_capacity]
  *   d_nnz       int32 [mask_heads]: kept blocks per mask head (always written)
+ *   d_row_order int32 [mask_heads][nq_blocks] or NULL: for each mask head the
+ *               query blocks ordered by decreasing row length (ties in
+ *               ascending order); bsattn_fwd_prefill uses it to start the
+ *               longest rows first
  *
  * When the kept blocks exceed col_capacity, no col_idx entry past the
  * capacity is written and *d_status (if given) receives BSATTN_ERR_CAPACITY;
@@ -105,7 +109,7 @@ int bsattn_debug_trace(int n, int32_t **host_view);
 int bsattn_build_index(const uint8_t *d_mask, int mask_heads, int nq_blocks, int nk_blocks,
                        int q_block, int k_block, int causal, int32_t *d_row_ptr,
                        int32_t *d_col_idx, int64_t col_capacity, int32_t *d_nnz,
-                       int32_t *d_status, cudaStream_t stream);
+                       int32_t *d_row_order, int32_t *d_status, cudaStream_t stream);
 
 /*
  * bsattn_fwd_prefill -- block-sparse attention over a whole sequence.
@@ -124,6 +128,9 @@ int bsattn_build_index(const uint8_t *d_mask, int mask_heads, int nq_blocks, int
  *   scale           softmax scale applied to Q K^T (e.g. 1/sqrt(d))
  *   row_ptr/col_idx CSR from bsattn_build_index (q_block = k_block = block),
  *                   or row_ptr = NULL for every tile
+ *   row_order       the builder's longest-first row order, or NULL; only the
+ *                   order in which query tiles are scheduled depends on it
+ *                   (BSATTN_ERR_INVALID_ARG when given without row_ptr)
  *   tile_status     uint8 [B][Hq][nq][nk] or NULL; the call first clears it,
  *                   then writes 1 for each visited-and-skipped tile and 2 for
  *                   each executed tile (0 = not visited)
@@ -134,8 +141,8 @@ int bsattn_build_index(const uint8_t *d_mask, int mask_heads, int nq_blocks, int
 int bsattn_fwd_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
                        int B, int Hq, int Hkv, int N, int d, int block, float scale, int causal,
                        float lambda, const int32_t *row_ptr, const int32_t *col_idx,
-                       int mask_heads, uint8_t *tile_status, int32_t *d_status,
-                       cudaStream_t stream);
+                       const int32_t *row_order, int mask_heads, uint8_t *tile_status,
+                       int32_t *d_status, cudaStream_t stream);
 
 /*
  * bsattn_decode_workspace_size -- bytes of scratch bsattn_fwd_decode needs:

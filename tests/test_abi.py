@@ -52,8 +52,8 @@ def _prefill(lib, q=0x1000, k=0x2000, v=0x3000, o=0x4000, B=1, Hq=2, Hkv=2, N=25
              block=128, scale=0.1, causal=0, lam=0.0, rp=None, ci=None, mh=1):
     return lib.bsattn_fwd_prefill(P(q) if q else None, P(k) if k else None, P(v) if v else None,
                                   P(o) if o else None, None, B, Hq, Hkv, N, d, block, scale,
-                                  causal, lam, P(rp) if rp else None, P(ci) if ci else None, mh,
-                                  None, None, None)
+                                  causal, lam, P(rp) if rp else None, P(ci) if ci else None, None,
+                                  mh, None, None, None)
 
 
 def test_prefill_host_validation(lib):
@@ -65,6 +65,9 @@ def test_prefill_host_validation(lib):
     assert _prefill(lib, scale=0.0) == -1
     assert _prefill(lib, rp=0x5000, ci=None) == -1   # CSR without col_idx
     assert _prefill(lib, rp=0x5000, ci=0x6000, mh=3) == -1
+    assert lib.bsattn_fwd_prefill(P(0x1000), P(0x2000), P(0x3000), P(0x4000), None, 1, 2, 2, 256,
+                                  128, 128, 0.1, 0, 0.0, None, None, P(0x7000), 1, None, None,
+                                  None) == -1           # row order without a CSR
     assert _prefill(lib, d=96) == -2                 # unsupported head dim
     assert _prefill(lib, block=32) == -2
     assert _prefill(lib, q=0x1001) == -3             # misaligned
@@ -93,11 +96,13 @@ def test_decode_host_validation(lib):
 
 def test_index_host_validation(lib):
     f = lib.bsattn_build_index
-    assert f(None, 1, 4, 4, 64, 64, 0, P(0x1000), P(0x2000), 16, P(0x3000), None, None) == -1
-    assert f(P(0x10), 0, 4, 4, 64, 64, 0, P(0x1000), P(0x2000), 16, P(0x3000), None, None) == -1
-    assert f(P(0x10), 1, 4, 4, 64, 64, 0, P(0x1000), P(0x2000), -1, P(0x3000), None, None) == -1
+    assert f(None, 1, 4, 4, 64, 64, 0, P(0x1000), P(0x2000), 16, P(0x3000), None, None, None) == -1
+    assert f(P(0x10), 0, 4, 4, 64, 64, 0, P(0x1000), P(0x2000), 16, P(0x3000), None, None,
+             None) == -1
+    assert f(P(0x10), 1, 4, 4, 64, 64, 0, P(0x1000), P(0x2000), -1, P(0x3000), None, None,
+             None) == -1
     assert f(P(0x10), 4096, 4096, 4096, 64, 64, 0, P(0x1000), P(0x2000), 16, P(0x3000), None,
-             None) == -2
+             None, None) == -2
 
 
 def test_debug_hook_validation(lib):

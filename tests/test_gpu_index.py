@@ -17,10 +17,18 @@ def _ops():
 def _gpu_index(m, qb, kb, causal, capacity=None):
     ops = _ops()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    rp, ci, nnz = ops.bsattn_build_index(torch.as_tensor(m).cuda().contiguous(), qb, kb, causal,
-                                         capacity=capacity, status=status)
+    rp, ci, nnz, order = ops.bsattn_build_index(torch.as_tensor(m).cuda().contiguous(), qb, kb,
+                                                causal, capacity=capacity, status=status,
+                                                with_order=True)
     torch.cuda.synchronize()
-    return rp.cpu().numpy(), ci.cpu().numpy(), nnz.cpu().numpy(), status.item()
+    rp, order = rp.cpu().numpy(), order.cpu().numpy()
+    # the longest-first schedule: a stable sort of each head's rows by length
+    Hm, nq = m.shape[0], m.shape[1]
+    for h in range(Hm):
+        lengths = np.diff(rp[h * (nq + 1):(h + 1) * (nq + 1)])
+        expect = np.argsort(-lengths, kind="stable")
+        assert (order[h * nq:(h + 1) * nq] == expect).all()
+    return rp, ci.cpu().numpy(), nnz.cpu().numpy(), status.item()
 
 
 @pytest.mark.parametrize("name", ["tiny", "mmdit", "videodit"])

@@ -18,25 +18,29 @@ def _ops():
     return ops
 
 
-def _run_gpu(w, lam, mask=None, mask_heads=1):
+def _run_gpu(w, lam, mask=None, mask_heads=1, ordered=True):
+    """Index (with the longest-first row order unless `ordered` is False) and
+    prefill through the C ABI; returns (o, lse, tile_status)."""
     ops = _ops()
     q, k, v = w.q.cuda(), w.k.cuda(), w.v.cuda()
-    rp = ci = None
+    rp = ci = order = None
     if mask is not None:
         m = torch.as_tensor(mask, dtype=torch.uint8).cuda().contiguous()
-        rp, ci, _ = ops.bsattn_build_index(m, w.block, w.block, w.causal)
+        rp, ci, _, order = ops.bsattn_build_index(m, w.block, w.block, w.causal, with_order=True)
         mask_heads = m.shape[0]
+        if not ordered:
+            order = None
     st = torch.zeros(w.B, w.Hq, w.nq, w.nk, dtype=torch.uint8, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     o, lse = ops.bsattn_fwd_prefill(q, k, v, w.block, w.scale, w.causal, lam, rp, ci, mask_heads,
-                                    tile_status=st, status=status)
+                                    tile_status=st, status=status, row_order=order)
     torch.cuda.synchronize()
     assert status.item() == 0, ops.bsattn_status_string(status.item())
     return o, lse, st
 
 
-def _check(w, lam, mask=None, what=""):
-    o, lse, st = _run_gpu(w, lam, mask)
+def _check(w, lam, mask=None, what="", ordered=True):
+    o, lse, st = _run_gpu(w, lam, mask, ordered=ordered)
     ref = oracle.prefill(w.q, w.k, w.v, w.block, w.scale, w.causal, lam, mask=mask)
     compare_outputs(o, ref["o"], lse, ref["lse"], what)
     compare_status(st, ref["status"], ref["margin"], what)
@@ -44,9 +48,10 @@ def _check(w, lam, mask=None, what=""):
 
 
 @pytest.mark.parametrize("name", ["tiny", "mmdit", "videodit"])
-def test_static_mask_workloads_shrunk(name):
+@pytest.mark.parametrize("ordered", [True, False])
+def test_static_mask_workloads_shrunk(name, ordered):
     w = inputs.workload(name, shrink=True)
-    _check(w, 0.0, w.mask.numpy(), name)
+    _check(w, 0.0, w.mask.numpy(), name, ordered=ordered)
 
 
 def test_mmdit_full_size():
