@@ -131,8 +131,9 @@ class ClockSampler:
 # ------------------------------------------------------------------ workloads
 def make_inputs(rank: int, a: float):
     from block_sparse_attention_bsattn_b200 import inputs
-    pw = inputs.workload("blasst_prefill", device="cuda", seed=1237 + 1000 * rank)
-    dw = inputs.workload("blasst_decode", device="cuda", seed=1238 + 1000 * rank)
+    ps, ds = rank_seeds(rank)
+    pw = inputs.workload("blasst_prefill", device="cuda", seed=ps)
+    dw = inputs.workload("blasst_decode", device="cuda", seed=ds)
     mask = torch.ones(1, pw.nq, pw.nk, dtype=torch.uint8, device="cuda")
     return pw, dw, mask
 
@@ -234,20 +235,38 @@ def timed_phases(step: Step, steps: int, phases=("index", "prefill", "decode")):
     return per, t0.elapsed_time(t1)
 
 
+def _reduce_device():
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
+
+
 def max_over_ranks(x: float) -> float:
+    """Largest value over all ranks (times: the slowest rank sets the step)."""
     if dist.is_initialized():
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=_reduce_device())
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
     return x
 
 
 def sum_over_ranks(x: float) -> float:
+    """Sum over all ranks (work: every rank processes its own units)."""
     if dist.is_initialized():
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=_reduce_device())
         dist.all_reduce(t, op=dist.ReduceOp.SUM)
         return float(t.item())
     return x
+
+
+def rank_seeds(rank: int):
+    """Seeds of the prefill and decode inputs of one rank: each rank draws its
+    own batch of the same workload (weak scaling)."""
+    return 1237 + 1000 * rank, 1238 + 1000 * rank
+
+
+def whole_job_rate(units_this_rank: float, ms_this_rank: float) -> float:
+    """Units per second of the whole job: all ranks' units over the slowest
+    rank's time."""
+    return sum_over_ranks(units_this_rank) / (max_over_ranks(ms_this_rank) * 1e-3)
 
 
 def barrier():

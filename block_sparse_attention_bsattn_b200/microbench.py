@@ -3,6 +3,12 @@
     python -m block_sparse_attention_bsattn_b200.microbench prefill --heads 8 --n 8192 --a 10
     python -m block_sparse_attention_bsattn_b200.microbench decode --batch 8 --a 10
     python -m block_sparse_attention_bsattn_b200.microbench videodit --heads 4
+    python -m block_sparse_attention_bsattn_b200.microbench table4
+
+`table4` sweeps lambda = a / L on the B200 shapes of the BLASST page's Table 4
+(prefill: batch 148, 1 query / 1 KV head, 32K tokens, d 128, causal; decode:
+batch 148, 32 query / 4 KV heads, 32K tokens, d 128) and reports, per a, the
+skipped fraction and the speed-up over the same kernel with lambda = 0.
 
 Used for Nsight Compute captures of a single kernel on a small case (a few
 launches, a few hundred MB on the device) and for quick CUDA-event timings.
@@ -31,9 +37,60 @@ def _time(fn, iters):
     return s.elapsed_time(e) / iters
 
 
+def table4(args):
+    rows = []
+    a_list = (0.0, 0.1, 1.0, 10.0, 100.0, 1000.0)
+    # prefill: B148 H1 N32768 d128 causal (one query head per KV head)
+    B, N = 148, 32768
+    q, k, v = inputs.blasst_prefill_qkv(B, 1, 1, N, 128, "cuda", 4242)
+    o = torch.empty_like(q)
+    nq = N // 128
+    base = None
+    for a in a_list:
+        lam = inputs.lambda_for(a, N)
+        st = torch.zeros(B, 1, nq, nq, dtype=torch.uint8, device="cuda")
+        ops.bsattn_fwd_prefill(q, k, v, 128, None, True, lam, o=o, tile_status=st, want_lse=False)
+        torch.cuda.synchronize()
+        vis, exe = int((st > 0).sum()), int((st == 2).sum())
+        fn = lambda: ops.bsattn_fwd_prefill(q, k, v, 128, None, True, lam, o=o, want_lse=False)
+        for _ in range(args.warmup):
+            fn()
+        ms = _time(fn, args.iters)
+        base = ms if base is None else base
+        rows.append({"kernel": "prefill", "a": a, "skipped": 1 - exe / vis, "ms": ms,
+                     "speedup_vs_dense": base / ms, "tflops": TILE * (vis + exe) / ms / 1e9})
+    del q, k, v, o
+    torch.cuda.empty_cache()
+    # decode: B148 Hq32/Hkv4 L32768 d128, 16 splits
+    B, Hq, Hkv, L = 148, 32, 4, 32768
+    q, k, v = inputs.blasst_decode_qkv(B, Hq, Hkv, L, 128, "cuda", 4243)
+    T = L // 128
+    ws = torch.empty(ops.bsattn_decode_workspace_size(B, Hq, 128, 16), dtype=torch.uint8,
+                     device="cuda")
+    o = torch.empty_like(q)
+    base = None
+    for a in a_list:
+        lam = inputs.lambda_for(a, L)
+        st = torch.zeros(B, Hkv, T, dtype=torch.uint8, device="cuda")
+        ops.bsattn_fwd_decode(q, k, v, 128, 16, None, lam, o=o, workspace=ws, tile_status=st,
+                              want_lse=False)
+        torch.cuda.synchronize()
+        vis, exe = int((st > 0).sum()), int((st == 2).sum())
+        fn = lambda: ops.bsattn_fwd_decode(q, k, v, 128, 16, None, lam, o=o, want_lse=False,
+                                           workspace=ws)
+        for _ in range(args.warmup):
+            fn()
+        ms = _time(fn, args.iters)
+        base = ms if base is None else base
+        byt = 2 * B * Hq * 128 * 2 + 128 * 128 * 2 * (vis + exe)
+        rows.append({"kernel": "decode", "a": a, "skipped": 1 - exe / vis, "ms": ms,
+                     "speedup_vs_dense": base / ms, "gbs": byt / ms / 1e6})
+    return rows
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=("prefill", "decode", "videodit", "mmdit"))
+    ap.add_argument("what", choices=("prefill", "decode", "videodit", "mmdit", "table4"))
     ap.add_argument("--heads", type=int, default=8, help="query heads (prefill/videodit/mmdit)")
     ap.add_argument("--n", type=int, default=32768, help="sequence length (prefill)")
     ap.add_argument("--batch", type=int, default=64, help="batch (decode)")
@@ -75,6 +132,8 @@ def main():
         tiles = int(nnz.sum()) * args.heads
         flops = 4 * w.block * w.block * w.d * tiles
         out.update(heads=args.heads, n=w.N, d=w.d, tiles=tiles, ms=ms, tflops=flops / ms / 1e9)
+    elif args.what == "table4":
+        out["rows"] = table4(args)
     else:
         B, Hq, Hkv, L, d = args.batch, 32, 8, args.l, 128
         q, k, v = inputs.blasst_decode_qkv(B, Hq, Hkv, L, d, "cuda", 1238)

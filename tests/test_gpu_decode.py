@@ -65,6 +65,14 @@ def test_decode_shapes(d, block, g, splits):
     _check(q, k, v, block, splits, 1 / math.sqrt(d), 2e-3, what=f"d{d} b{block} g{g} s{splits}")
 
 
+@pytest.mark.parametrize("a", [0.0, 10.0, 1000.0])
+def test_decode_table4_shape_shrunk(a):
+    """32 query / 4 KV heads (group of 8), the BLASST page's Table 4 decode shape
+    with fewer sequences and a shorter cache."""
+    q, k, v = inputs.blasst_decode_qkv(3, 32, 4, 8192, 128, "cpu", 4243)
+    _check(q, k, v, 128, 16, 1 / math.sqrt(128), inputs.lambda_for(a, 8192), what=f"t4 a={a}")
+
+
 def test_more_splits_than_tiles():
     q, k, v = inputs.blasst_decode_qkv(1, 4, 1, 300, 128, "cpu", 9)
     _check(q, k, v, 128, 8, 1 / math.sqrt(128), 1e-2, what="empty splits")

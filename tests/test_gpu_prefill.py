@@ -101,6 +101,18 @@ def test_blasst_random_masks_per_head(d, block):
     assert torch.isneginf(lse[:, :, rows]).all()
 
 
+@pytest.mark.parametrize("a", [0.0, 10.0, 1000.0])
+def test_blasst_prefill_one_head_per_kv_head(a):
+    """Causal BLASST prefill with one query head per KV head and several
+    sequences (the shape of the BLASST page's Table 4 prefill, shrunk): the
+    single-query-tile kernel."""
+    B, H, N = 3, 1, 2048 + 96
+    q, k, v = inputs.blasst_prefill_qkv(B, H, H, N, 128, "cpu", 4242)
+    w = inputs.Workload("t4", B, H, H, N, 128, 128, True, "prefill", 1 / math.sqrt(128), None,
+                        q=q, k=k, v=v)
+    _check(w, inputs.lambda_for(a, N), None, f"table4-shape a={a}")
+
+
 def test_short_sequence_single_partial_tile():
     q, k, v = inputs.normal_qkv(1, 2, 2, 50, 128, "cpu", 3)
     w = inputs.Workload("short", 1, 2, 2, 50, 128, 128, True, "prefill", 1 / math.sqrt(128), None,
