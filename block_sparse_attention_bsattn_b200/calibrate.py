@@ -77,13 +77,24 @@ def main():
     ap.add_argument("--tol", type=float, default=0.05)
     ap.add_argument("--lengths", default="4096,8192,16384,32768")
     ap.add_argument("--heads", type=int, default=8)
-    ap.add_argument("--lambdas", type=int, default=25, help="log grid size over [1e-7, 1e-1]")
+    ap.add_argument("--lambdas", type=int, default=31, help="log grid size over [1e-10, 1]")
     args = ap.parse_args()
     lengths = [int(x) for x in args.lengths.split(",")]
-    lambdas = log_grid(1e-7, 1e-1, args.lambdas)
+    lambdas = log_grid(1e-10, 1.0, args.lambdas)
     cache: dict = {}
-    measure = lambda lam, L: prefill_sparsity(lam, L, heads=args.heads, cache=cache)
-    a, points = calibrate(measure, lengths, lambdas, args.target, args.tol)
+    curve: dict = {}
+
+    def measure(lam, L):
+        s = prefill_sparsity(lam, L, heads=args.heads, cache=cache)
+        curve.setdefault(L, []).append((lam, s))
+        return s
+
+    try:
+        a, points = calibrate(measure, lengths, lambdas, args.target, args.tol)
+    except ValueError as e:
+        print(json.dumps({"target": args.target, "error": str(e),
+                          "measured": {str(L): c for L, c in curve.items()}}), flush=True)
+        raise SystemExit(2)
     # achieved sparsity of the fitted law at every length
     check = [{"L": L, "lambda": a / L, "sparsity": measure(a / L, L)} for L in lengths]
     print(json.dumps({"target": args.target, "tol": args.tol, "a": a,

@@ -207,12 +207,16 @@ int bsattn_fwd_prefill(const void* q, const void* k, const void* v, void* o, flo
   p.trace_n = g_trace_n;
 
   cudaError_t e;
-  // Two query heads of one KV head share a CTA and its K/V stream when the
-  // group size is even and both heads walk the same visit list.
-  const bool pair = block == 128 && (Hq / Hkv) % 2 == 0 && (!row_ptr || mask_heads == 1);
-  if (pair) {
-    e = d == 128 ? launch_prefill_pair<128>(tq, tk, tv, p, (int)(items / 2), stream)
-                 : launch_prefill_pair<64>(tq, tk, tv, p, (int)(items / 2), stream);
+  // Two query tiles share a CTA and its K/V stream when they walk the same
+  // visit list: two query heads of one KV head (group size even), or, without
+  // a block mask, two consecutive query tiles of one head.
+  const bool pair_heads = block == 128 && (Hq / Hkv) % 2 == 0 && (!row_ptr || mask_heads == 1);
+  const bool pair_tiles = block == 128 && !pair_heads && !row_ptr;
+  if (pair_heads || pair_tiles) {
+    p.pair_tiles = pair_tiles ? 1 : 0;
+    const int64_t pitems = pair_heads ? items / 2 : (int64_t)B * Hq * ((nq + 1) / 2);
+    e = d == 128 ? launch_prefill_pair<128>(tq, tk, tv, p, (int)pitems, stream)
+                 : launch_prefill_pair<64>(tq, tk, tv, p, (int)pitems, stream);
     return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
   }
   if (d == 128 && block == 128) e = launch_prefill<128, 128>(tq, tk, tv, p, (int)items, stream);

@@ -32,7 +32,8 @@ struct PrefillParams {
   float scale_log2;  // softmax scale * log2(e): scores are kept in base-2 units
   float thr_log2;    // log2(lambda)
   int use_skip;      // lambda > 0
-  int debug_stall;   // test hook: the producer never issues the Q load
+  int debug_stall;   // test hook: the query tile is withheld from the tensor core
+  int pair_tiles;    // two-slot kernel: consecutive query tiles of one head
   unsigned long long wait_limit_ns;
   volatile int32_t* trace;  // debug: progress markers (host-visible memory) or null
   int trace_n;

@@ -1,6 +1,10 @@
-// Block-sparse prefill for two query heads that share a KV head (GQA group of
-// even size): one CTA runs the same query tile of both heads against one K/V
-// stream, so every K and V tile crosses L2 once for two query tiles.
+// Block-sparse prefill for two query tiles that walk the same K/V stream, so
+// every K and V tile crosses L2 once for two query tiles:
+//   heads mode  the same query tile of two query heads that share a KV head
+//               (GQA group of even size, one visit list for the group);
+//   tiles mode  two consecutive query tiles of one head when no block mask is
+//               given (every key tile, or the causal prefix, which differs by
+//               the diagonal tile only): slot e visits stream tiles t < n_e.
 //
 // Same method as prefill_sm100.cu ("BLASST: Dynamic Blocked Attention Sparsity
 // via Softmax Thresholding", Algorithm 1 and section 4.1; "块稀疏Attention实战"
@@ -85,37 +89,60 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // ---- work item: (batch, head pair, query tile); heads 2*pr and 2*pr + 1
-  // share KV head (2*pr) / group
-  const int PH = p.Hq / 2;
-  const int BP = p.B * PH;
-  int i, bp;
-  if (p.row_order) {
-    bp = (int)(blockIdx.x / p.nq);
-    i = p.row_order[(int)(blockIdx.x % p.nq)];
-  } else if (p.causal) {
-    i = p.nq - 1 - (int)(blockIdx.x / BP);
-    bp = (int)(blockIdx.x % BP);
-  } else {
-    bp = (int)(blockIdx.x / p.nq);
-    i = (int)(blockIdx.x % p.nq);
-  }
-  const int b = bp / PH, h0 = 2 * (bp % PH);
-  const int kvh = h0 / (p.Hq / p.Hkv);
-
-  // ---- visit list (mask head 0: both heads share it)
+  // ---- work item -> two slots (head h_e, query tile i_e, visit length n_e)
+  int b, hs[2], is[2], ns[2];
   const int32_t* cols = nullptr;
-  int n;
-  if (p.row_ptr) {
-    const int32_t s0 = p.row_ptr[i];
-    const int32_t s1 = p.row_ptr[i + 1];
-    cols = p.col_idx + s0;
-    n = s1 - s0;
-    if (p.causal)
-      while (n > 0 && cols[n - 1] > i) --n;
+  int n;  // length of the shared K/V stream
+  if (!p.pair_tiles) {
+    const int PH = p.Hq / 2;
+    const int BP = p.B * PH;
+    int i, bp;
+    if (p.row_order) {
+      bp = (int)(blockIdx.x / p.nq);
+      i = p.row_order[(int)(blockIdx.x % p.nq)];
+    } else if (p.causal) {
+      i = p.nq - 1 - (int)(blockIdx.x / BP);
+      bp = (int)(blockIdx.x % BP);
+    } else {
+      bp = (int)(blockIdx.x / p.nq);
+      i = (int)(blockIdx.x % p.nq);
+    }
+    b = bp / PH;
+    hs[0] = 2 * (bp % PH);
+    hs[1] = hs[0] + 1;
+    is[0] = is[1] = i;
+    // visit list of mask head 0, shared by both heads
+    if (p.row_ptr) {
+      const int32_t s0 = p.row_ptr[i];
+      const int32_t s1 = p.row_ptr[i + 1];
+      cols = p.col_idx + s0;
+      n = s1 - s0;
+      if (p.causal)
+        while (n > 0 && cols[n - 1] > i) --n;
+    } else {
+      n = p.causal ? i + 1 : p.nk;
+    }
+    ns[0] = ns[1] = n;
   } else {
-    n = p.causal ? i + 1 : p.nk;
+    const int NP = (p.nq + 1) / 2;
+    const int BH = p.B * p.Hq;
+    int m, bh;
+    if (p.causal) {                       // longest pairs first
+      m = NP - 1 - (int)(blockIdx.x / BH);
+      bh = (int)(blockIdx.x % BH);
+    } else {
+      bh = (int)(blockIdx.x / NP);
+      m = (int)(blockIdx.x % NP);
+    }
+    b = bh / p.Hq;
+    hs[0] = hs[1] = bh % p.Hq;
+    is[0] = 2 * m;
+    is[1] = 2 * m + 1;
+    ns[0] = p.causal ? is[0] + 1 : p.nk;
+    ns[1] = is[1] < p.nq ? (p.causal ? is[1] + 1 : p.nk) : 0;
+    n = max(ns[0], ns[1]);
   }
+  const int kvh = hs[0] / (p.Hq / p.Hkv);
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -157,7 +184,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int e = 0; e < 2; ++e)
           for (int hf = 0; hf < C::HALVES; ++hf)
             tma_load_3d(q_smem + e * C::Q_BYTES + hf * C::Q_HALF, &tmQ, &bars->q_full, hf * 64,
-                        i * BLK, b * p.Hq + h0 + e);
+                        is[e] * BLK, b * p.Hq + hs[e]);
       }
       int issued_k = 0, issued_v = 0;
       for (int t = 0; t < n; ++t) {
@@ -222,8 +249,8 @@ __global__ void __launch_bounds__(320, 1)
         ok = mbar_wait(&bars->k_full[0], 0, abort, lim);
         tc_fence_after();
         if (ok) {
-          bmm1(0, 0);
-          bmm1(1, 0);
+          if (ns[0] > 0) bmm1(0, 0);
+          if (ns[1] > 0) bmm1(1, 0);
           mma_commit(&bars->k_empty[0]);
         }
       }
@@ -231,9 +258,11 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = 0; ok && t < n; ++t) {
         const int vs = t % C::VST;
         bool v_ready = false;
+        bool k_next = false;        // K_{t+1} waited for
         const bool more = t + 1 < n;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
+          if (t >= ns[e]) continue;  // this slot's visit list is shorter
           if (!mbar_wait(&bars->p_ready[e], t & 1, abort, lim)) { ok = false; break; }
           tc_fence_after();
           const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[e]);
@@ -246,11 +275,12 @@ __global__ void __launch_bounds__(320, 1)
             bmm2(e, t, kept[e] == 0);
             ++kept[e];
           }
-          if (more) {
-            if (e == 0) {   // first use of K_{t+1}
+          if (t + 1 < ns[e]) {
+            if (!k_next) {   // first use of K_{t+1}
               const int ks = (t + 1) % C::KST;
               if (!mbar_wait(&bars->k_full[ks], ((t + 1) / C::KST) & 1, abort, lim)) { ok = false; break; }
               tc_fence_after();
+              k_next = true;
             }
             bmm1(e, t + 1);
           }
@@ -270,19 +300,21 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     // ======================================================== softmax warps
-    const int e = (warp - 2) / 4;           // which head of the pair
+    const int e = (warp - 2) / 4;           // which slot of the pair
     const int sw = (warp - 2) % 4;
     const int quarter = warp % 4;
     const int row = quarter * 32 + lane;
+    const int i = is[e];
     const int r0 = i * BLK;
-    const int h = h0 + e;
+    const int h = hs[e];
+    const int ne = ns[e];
     const bool valid = r0 + row < p.N;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t s_col = 256 * e, o_col = 256 * e + 128;
     float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
     int kept = 0;
     bool ok = true;
-    for (int t = 0; t < n; ++t) {
+    for (int t = 0; t < ne; ++t) {
       const int j = cols ? cols[t] : t;
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[e], t & 1, abort, lim))) {
         ok = false;

@@ -1,0 +1,42 @@
+"""Failure detection without a GPU fault: a test switch makes the prefill
+kernel withhold its query tile, so one pipeline wait runs out (a short limit).
+The kernel must drain its own copies, free its tensor memory, return, and
+report BSATTN_ERR_DEVICE_TIMEOUT in the status word; the context must stay
+usable (a normal call afterwards is correct).  Nothing traps, faults or
+hangs."""
+import math
+
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_bsattn_b200 import inputs
+from tests.parity import compare_outputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _ops():
+    from block_sparse_attention_bsattn_b200 import ops
+    return ops
+
+
+@pytest.mark.parametrize("hq,hkv", [(2, 1), (1, 1)])   # two-head kernel, one-tile kernel
+def test_stalled_pipeline_reports_timeout_and_recovers(hq, hkv):
+    ops = _ops()
+    q, k, v = inputs.normal_qkv(1, hq, hkv, 256, 128, "cpu", 3)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        ops.bsattn_debug_set(50_000_000, inject_stall=True)   # 50 ms per wait
+        ops.bsattn_fwd_prefill(qd, kd, vd, 128, None, True, 0.0, status=status)
+        torch.cuda.synchronize()
+        assert status.item() == -6, ops.bsattn_status_string(status.item())
+    finally:
+        ops.bsattn_debug_set(2_000_000_000, inject_stall=False)
+    status.zero_()
+    o, lse = ops.bsattn_fwd_prefill(qd, kd, vd, 128, None, True, 0.0, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ref = oracle.prefill(q, k, v, 128, 1 / math.sqrt(128), True, 0.0)
+    compare_outputs(o, ref["o"], lse, ref["lse"], "after timeout")

@@ -70,9 +70,12 @@ def test_blasst_prefill_shrunk(a):
 
 @pytest.mark.parametrize("d,block", [(64, 64), (64, 128), (128, 64), (128, 128)])
 @pytest.mark.parametrize("causal", [False, True])
-def test_dense_shapes_and_tails(d, block, causal):
-    """Every (d, block) variant, causal and not, with a ragged tail and GQA 4."""
-    B, Hq, Hkv, N = 2, 4, 1, 3 * block + 37
+@pytest.mark.parametrize("hq,hkv,nt", [(4, 1, 3), (3, 3, 4)])
+def test_dense_shapes_and_tails(d, block, causal, hq, hkv, nt):
+    """Every (d, block) variant, causal and not, with a ragged tail; GQA 4
+    (head pairs share a CTA) and GQA 1 with an odd number of query tiles
+    (consecutive query tiles share a CTA, the last one alone)."""
+    B, Hq, Hkv, N = 2, hq, hkv, nt * block + 37
     q, k, v = inputs.normal_qkv(B, Hq, Hkv, N, d, "cpu", 100 + d + block)
     w = inputs.Workload("dense", B, Hq, Hkv, N, d, block, causal, "prefill", 1 / math.sqrt(d),
                         None, q=q, k=k, v=v)
