@@ -92,11 +92,16 @@ struct DecTcBarriers {
   int dec[8];        // decision queue: kept flag
 };
 
-template <int D>
+// NC: the query columns the softmax warps work on, G rounded up to a power of
+// two, fixed at compile time so that the per-column work of the scores (the
+// reduction, the vote, the exponentials) unrolls and interleaves
+template <int D, int NC>
 __global__ void __launch_bounds__(224, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const DecodeParams p, int G) {
   using C = DecTcCfg<D>;
+  static_assert(NC == 1 || NC == 2 || NC == 4 || NC == 8 || NC == 16, "columns");
+  constexpr int LOG_NC = NC >= 16 ? 4 : NC >= 8 ? 3 : NC >= 4 ? 2 : NC >= 2 ? 1 : 0;
   static_assert(sizeof(DecTcBarriers) <= C::BAR_BYTES, "barrier block");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -306,9 +311,9 @@ __global__ void __launch_bounds__(224, 1)
     for (int n = 0; ok && n < my_items; ++n) {
       int b, kvh, split, t0, nt;
       item_of(n, b, kvh, split, t0, nt);
-      float m_run[16], m_ref[16], lp[16];
+      float m_run[NC], m_ref[NC], lp[NC];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) { m_run[c] = -INFINITY; m_ref[c] = -INFINITY; lp[c] = 0.f; }
+      for (int c = 0; c < NC; ++c) { m_run[c] = -INFINITY; m_ref[c] = -INFINITY; lp[c] = 0.f; }
       int kept_item = 0;
       for (int t = 0; t < nt; ++t, ++g) {
         const int sb = g % C::NS;
@@ -330,37 +335,49 @@ __global__ void __launch_bounds__(224, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
         const bool key_ok = (t0 + t) * C::BLK + key < p.L;
-        float s[16];
+        float s[NC];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) s[c] = key_ok ? __uint_as_float(r[c]) : -INFINITY;
-        // tile max per query column: warp, then across the four warps
+        for (int c = 0; c < NC; ++c) s[c] = (key_ok && c < G) ? __uint_as_float(r[c]) : -INFINITY;
+        // tile max per query column.  Inside the warp a butterfly that halves
+        // the columns a lane holds at each exchange (NC - 1 shuffles, then a
+        // plain reduction over the remaining lane bits) leaves lane l with the
+        // maximum of column l >> (5 - log2 NC); across the four warps through
+        // one shared-memory slot per warp and column.
         float* rr = red + (g & 1) * 4 * C::NQ;
+        {
+          float v[NC];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          if (c >= G) break;
-          float m = s[c];
+          for (int c = 0; c < NC; ++c) v[c] = s[c];
 #pragma unroll
-          for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-          if (lane == 0) rr[sw * C::NQ + c] = m;
+          for (int k = 0; k < LOG_NC; ++k) {
+            const int w = NC >> (k + 1);
+            const bool up = (lane >> (4 - k)) & 1;
+#pragma unroll
+            for (int i = 0; i < w; ++i) {
+              const float send = up ? v[i] : v[i + w];
+              const float keep = up ? v[i + w] : v[i];
+              v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 16 >> k));
+            }
+          }
+#pragma unroll
+          for (int off = 16 >> LOG_NC; off > 0; off >>= 1)
+            v[0] = fmaxf(v[0], __shfl_xor_sync(0xffffffffu, v[0], off));
+          if ((lane & ((32 >> LOG_NC) - 1)) == 0) rr[sw * C::NQ + (lane >> (5 - LOG_NC))] = v[0];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->red_bar[g & 1]);
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->red_bar[g & 1], (g >> 1) & 1, abort, lim))) { ok = false; break; }
         bool all_pass = true;
-        float mt[16];
+        float mt[NC];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          if (c >= G) break;
+        for (int c = 0; c < NC; ++c) {
           const float m = fmaxf(fmaxf(rr[c], rr[C::NQ + c]), fmaxf(rr[2 * C::NQ + c], rr[3 * C::NQ + c]));
           mt[c] = m * p.scale_log2;
-          all_pass = all_pass && (mt[c] - m_run[c] < thr);
+          if (c < G) all_pass = all_pass && (mt[c] - m_run[c] < thr);
         }
         const bool skip = p.use_skip && all_pass;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          if (c >= G) break;
-          m_run[c] = fmaxf(m_run[c], mt[c]);
-        }
+        for (int c = 0; c < NC; ++c) m_run[c] = fmaxf(m_run[c], mt[c]);
         // the decision goes to the V producer and (for tile status) to memory
         if (sw == 0 && lane == 0) {
           const int dq = g % C::DQ;
@@ -382,8 +399,9 @@ __global__ void __launch_bounds__(224, 1)
           bool rescale = false;
           float alpha[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            alpha[c] = 1.f;
+          for (int c = 0; c < 16; ++c) alpha[c] = 1.f;
+#pragma unroll
+          for (int c = 0; c < NC; ++c) {
             if (c >= G) continue;
             if (kept_item == 0) {
               m_ref[c] = m_run[c];
@@ -412,13 +430,12 @@ __global__ void __launch_bounds__(224, 1)
             tmem_st16(lane_addr + C::O_COL + (n & 1) * 16, o);
             tmem_wait_st();
 #pragma unroll
-            for (int c = 0; c < 16; ++c) lp[c] *= alpha[c];
+            for (int c = 0; c < NC; ++c) lp[c] *= alpha[c];
           }
           // P^T[c][key] = exp2(S * scale_log2 - shift) as bf16, 128-byte swizzle
           uint8_t* ps = p_smem + (kept % C::PB) * C::P_BYTES + (key / 64) * C::P_HALF;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            if (c >= G) break;
+          for (int c = 0; c < NC; ++c) {
             const float sh = m_ref[c] == -INFINITY ? 0.f : m_ref[c];
             const float pv = fast_exp2(fmaf(s[c], p.scale_log2, -sh));
             lp[c] += pv;
@@ -463,7 +480,7 @@ __global__ void __launch_bounds__(224, 1)
         break;
       }
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
+      for (int c = 0; c < NC; ++c) {
         if (c >= G) break;
         float x = lp[c];
 #pragma unroll
@@ -490,7 +507,7 @@ __global__ void __launch_bounds__(224, 1)
           const float l = rl[lane] + rl[C::NQ + lane] + rl[2 * C::NQ + lane] + rl[3 * C::NQ + lane];
           float mr = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
+          for (int c = 0; c < NC; ++c)
             if (c == lane) mr = m_ref[c];
           p.ws_l[base + (int64_t)lane * p.splits] = kept_item > 0 ? l : 0.f;
           p.ws_m[base + (int64_t)lane * p.splits] = kept_item > 0 ? mr : -INFINITY;
@@ -510,16 +527,27 @@ __global__ void __launch_bounds__(224, 1)
   }
 }
 
+template <int D, int NC>
+static cudaError_t launch_decode_tc_nc(const CUtensorMap& tq, const CUtensorMap& tk,
+                                       const CUtensorMap& tv, const DecodeParams& p, int G, int grid,
+                                       cudaStream_t stream) {
+  using C = DecTcCfg<D>;
+  static_assert(C::SMEM <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, NC>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  decode_tc_kernel<D, NC><<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p, G);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_decode_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const DecodeParams& p, int G, int grid, cudaStream_t stream) {
-  using C = DecTcCfg<D>;
-  static_assert(C::SMEM <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return e;
-  decode_tc_kernel<D><<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p, G);
-  return cudaGetLastError();
+  if (G <= 1) return launch_decode_tc_nc<D, 1>(tq, tk, tv, p, G, grid, stream);
+  if (G <= 2) return launch_decode_tc_nc<D, 2>(tq, tk, tv, p, G, grid, stream);
+  if (G <= 4) return launch_decode_tc_nc<D, 4>(tq, tk, tv, p, G, grid, stream);
+  if (G <= 8) return launch_decode_tc_nc<D, 8>(tq, tk, tv, p, G, grid, stream);
+  return launch_decode_tc_nc<D, 16>(tq, tk, tv, p, G, grid, stream);
 }
 
 template cudaError_t launch_decode_tc<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,

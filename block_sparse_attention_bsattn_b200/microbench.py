@@ -95,6 +95,8 @@ def main():
     ap.add_argument("--n", type=int, default=32768, help="sequence length (prefill)")
     ap.add_argument("--batch", type=int, default=64, help="batch (decode)")
     ap.add_argument("--l", type=int, default=131072, help="KV length (decode)")
+    ap.add_argument("--hkv", type=int, default=8, help="KV heads (decode; 32 query heads)")
+    ap.add_argument("--splits", type=int, default=16, help="KV splits (decode)")
     ap.add_argument("--a", type=float, default=10.0)
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=2)
@@ -135,23 +137,24 @@ def main():
     elif args.what == "table4":
         out["rows"] = table4(args)
     else:
-        B, Hq, Hkv, L, d = args.batch, 32, 8, args.l, 128
+        B, Hq, Hkv, L, d = args.batch, 32, args.hkv, args.l, 128
+        ns = args.splits
         q, k, v = inputs.blasst_decode_qkv(B, Hq, Hkv, L, d, "cuda", 1238)
         lam = inputs.lambda_for(args.a, L)
         T = -(-L // 128)
         st = torch.zeros(B, Hkv, T, dtype=torch.uint8, device="cuda")
-        ws = torch.empty(ops.bsattn_decode_workspace_size(B, Hq, d, 16), dtype=torch.uint8,
+        ws = torch.empty(ops.bsattn_decode_workspace_size(B, Hq, d, ns), dtype=torch.uint8,
                          device="cuda")
-        o, _ = ops.bsattn_fwd_decode(q, k, v, 128, 16, None, lam, workspace=ws, tile_status=st)
+        o, _ = ops.bsattn_fwd_decode(q, k, v, 128, ns, None, lam, workspace=ws, tile_status=st)
         torch.cuda.synchronize()
         vis, exe = int((st > 0).sum()), int((st == 2).sum())
-        fn = lambda: ops.bsattn_fwd_decode(q, k, v, 128, 16, None, lam, o=o, want_lse=False,
+        fn = lambda: ops.bsattn_fwd_decode(q, k, v, 128, ns, None, lam, o=o, want_lse=False,
                                            workspace=ws)
         for _ in range(args.warmup):
             fn()
         ms = _time(fn, args.iters)
         byt = 2 * B * Hq * d * 2 + 128 * d * 2 * (vis + exe)
-        out.update(batch=B, l=L, a=args.a, visited=vis, executed=exe, ms=ms, gbs=byt / ms / 1e6)
+        out.update(batch=B, l=L, hkv=Hkv, splits=ns, a=args.a, visited=vis, executed=exe, ms=ms, gbs=byt / ms / 1e6)
     print(json.dumps(out), flush=True)
 
 
