@@ -532,10 +532,10 @@ def main():
                     "strict_flops_per_launch": strict_flops,
                     "strict_tflops": strict_flops / (p_ms * 1e-3) / 1e12,
                     "launch_ms": p_ms}
-    decode_roof = {"kernel": "decode_tc_kernel<128> + decode_combine_kernel",
+    decode_roof = {"kernel": "decode_tc_kernel<128, 4> + decode_combine_kernel",
                    "bound": "hbm", "achieved": gb_rank, "peak": hbm_peak,
                    "unit": "GB/s", "frac": gb_rank / hbm_peak,
-                   "traffic": profiled_traffic("decode_tc_kernel<128>"),
+                   "traffic": profiled_traffic("decode_tc_kernel<128, 4>"),
                    "peak_source": f"{peak_src} copy bandwidth",
                    "bytes_per_launch": d_bytes, "launch_ms": d_ms}
     # the top-level roofline is the one of the kernel that takes the larger

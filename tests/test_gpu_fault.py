@@ -21,22 +21,24 @@ def _ops():
     return ops
 
 
-@pytest.mark.parametrize("hq,hkv", [(2, 1), (1, 1)])   # two-head kernel, one-tile kernel
-def test_stalled_pipeline_reports_timeout_and_recovers(hq, hkv):
+# two heads of one KV head (pair kernel, heads mode), one head (pair kernel,
+# two consecutive query tiles), 64-token tiles (one-query-tile kernel)
+@pytest.mark.parametrize("hq,hkv,block", [(2, 1, 128), (1, 1, 128), (1, 1, 64)])
+def test_stalled_pipeline_reports_timeout_and_recovers(hq, hkv, block):
     ops = _ops()
     q, k, v = inputs.normal_qkv(1, hq, hkv, 256, 128, "cpu", 3)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     try:
         ops.bsattn_debug_set(50_000_000, inject_stall=True)   # 50 ms per wait
-        ops.bsattn_fwd_prefill(qd, kd, vd, 128, None, True, 0.0, status=status)
+        ops.bsattn_fwd_prefill(qd, kd, vd, block, None, True, 0.0, status=status)
         torch.cuda.synchronize()
         assert status.item() == -6, ops.bsattn_status_string(status.item())
     finally:
         ops.bsattn_debug_set(2_000_000_000, inject_stall=False)
     status.zero_()
-    o, lse = ops.bsattn_fwd_prefill(qd, kd, vd, 128, None, True, 0.0, status=status)
+    o, lse = ops.bsattn_fwd_prefill(qd, kd, vd, block, None, True, 0.0, status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
-    ref = oracle.prefill(q, k, v, 128, 1 / math.sqrt(128), True, 0.0)
+    ref = oracle.prefill(q, k, v, block, 1 / math.sqrt(128), True, 0.0)
     compare_outputs(o, ref["o"], lse, ref["lse"], "after timeout")
