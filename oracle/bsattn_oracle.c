@@ -29,10 +29,17 @@
  *    running max passes.
  *  - The running max is updated with every visited tile, skipped or not
  *    (Algorithm 1 updates it before the test).
- *  - Visit order is ascending key-tile index.
+ *  - Visit order is ascending key-tile index (Algorithm 1's loop over j), or,
+ *    on request, descending: the BLASST page's block-row reordering study
+ *    (section on ablations, Figure 8) visits the tiles of a row in reverse so
+ *    that the local window, which holds the largest scores, sets the running
+ *    max first.
  *  - Decode: the query tile is the g query heads that share one KV head; the
  *    KV tiles are cut into num_splits contiguous chunks of ceil(T/num_splits)
- *    tiles and the running max starts again at -inf in each chunk.
+ *    tiles and the running max starts again at -inf in each chunk.  On
+ *    request (sink seeding) every chunk but the first starts instead from the
+ *    row max of key tile 0, the tile that holds the attention sink; tile 0 is
+ *    then scored by that chunk but neither visited nor executed by it.
  *  - The result is the exact softmax over the keys of the executed tiles,
  *    computed in two passes (max, then sum) -- algebraically what the online
  *    recurrence of Algorithm 1 reaches.
@@ -121,11 +128,14 @@ int oracle_build_index(const uint8_t *mask, int mask_heads, int nq, int nk,
  *   status: per visited tile, 1 = skipped, 2 = executed
  *   margin: per visited tile, max over rows of (tile max - running max)
  *           minus ln(lambda); +inf when the test cannot pass
+ *   seed_tile: -1, or a key tile whose row max starts the running max at every
+ *           split start whose first tile is another tile
  */
 static void query_tile(const uint16_t *const *qrows, const int64_t *qpos, int nrows,
                        const uint16_t *kbase, const uint16_t *vbase, int64_t L,
                        int d, int block, double scale, int causal, double lambda,
                        const int32_t *tiles, const uint8_t *split_start, int ntiles,
+                       int seed_tile,
                        double *out, double *lse, uint8_t *status, double *margin)
 {
     const double ln_lambda = lambda > 0.0 ? log(lambda) : -INFINITY;
@@ -169,9 +179,17 @@ static void query_tile(const uint16_t *const *qrows, const int64_t *qpos, int nr
     for (int r = 0; r < nrows; ++r)
         mprev[r] = -INFINITY;
     for (int t = 0; t < ntiles; ++t) {
-        if (split_start && split_start[t])
+        if (split_start && split_start[t]) {
             for (int r = 0; r < nrows; ++r)
                 mprev[r] = -INFINITY;
+            if (seed_tile >= 0 && tiles[t] != seed_tile) {
+                SCORE_TILE(seed_tile);
+                for (int r = 0; r < nrows; ++r)
+                    for (int c = 0; c < block; ++c)
+                        if (s[(size_t)r * block + c] > mprev[r])
+                            mprev[r] = s[(size_t)r * block + c];
+            }
+        }
         SCORE_TILE(tiles[t]);
         double dmax = -INFINITY;
         for (int r = 0; r < nrows; ++r) {
@@ -261,13 +279,15 @@ static void query_tile(const uint16_t *const *qrows, const int64_t *qpos, int nr
  * items: NULL (every (b, h, i)) or n_items triples (b, h, i) to compute.
  * o: [B][Hq][N][d], lse: [B][Hq][N] (doubles); tile_status / margin:
  * NULL or [B][Hq][nq][nk].  Only rows of the listed items are written.
+ * reverse: 0 visits each row's key tiles in ascending order, 1 in descending.
  */
 int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                    int B, int Hq, int Hkv, int N, int d, int block,
                    double scale, int causal, double lambda,
                    const uint8_t *mask, int mask_heads,
                    const int32_t *items, int n_items,
-                   double *o, double *lse, uint8_t *tile_status, double *margin)
+                   double *o, double *lse, uint8_t *tile_status, double *margin,
+                   int reverse)
 {
     if (!q || !k || !v || !o || !lse || B < 1 || Hq < 1 || Hkv < 1 ||
         Hq % Hkv != 0 || N < 1 || d < 1 || block < 1 ||
@@ -310,6 +330,12 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 continue;
             tiles[nt++] = j;
         }
+        if (reverse)
+            for (int a = 0, z = nt - 1; a < z; ++a, --z) {
+                int32_t x = tiles[a];
+                tiles[a] = tiles[z];
+                tiles[z] = x;
+            }
         uint8_t *st = malloc(nt > 0 ? nt : 1);
         double *mg = malloc(sizeof(double) * (nt > 0 ? nt : 1));
         const uint16_t *kb = k + ((int64_t)b * Hkv + kvh) * N * d;
@@ -317,7 +343,7 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         double *orow = o + (((int64_t)b * Hq + h) * N + r0) * d;
         double *lrow = lse + ((int64_t)b * Hq + h) * N + r0;
         query_tile(qrows, qpos, nrows, kb, vb, N, d, block, scale, causal, lambda,
-                   tiles, NULL, nt, orow, lrow, st, mg);
+                   tiles, NULL, nt, -1, orow, lrow, st, mg);
         int64_t sbase = (((int64_t)b * Hq + h) * nq + i) * nk;
         for (int t = 0; t < nt; ++t) {
             if (tile_status)
@@ -337,11 +363,13 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
  * q: [n][g][d] (the g query heads sharing the KV head), k, v: [n][L][d].
  * o: [n][g][d], lse: [n][g]; tile_status / margin: NULL or [n][T] with
  * T = ceil(L / block).  A single query at the last position sees all L keys.
+ * sink_seed: 1 starts every split after the first from key tile 0's row max.
  */
 int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                   int n_problems, int g, int64_t L, int d, int block,
                   double scale, double lambda, int num_splits,
-                  double *o, double *lse, uint8_t *tile_status, double *margin)
+                  double *o, double *lse, uint8_t *tile_status, double *margin,
+                  int sink_seed)
 {
     if (!q || !k || !v || !o || !lse || n_problems < 1 || g < 1 || g > 1024 ||
         L < 1 || d < 1 || block < 1 || num_splits < 1 ||
@@ -367,7 +395,7 @@ int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         uint8_t *st = malloc(T);
         double *mg = malloc(sizeof(double) * T);
         query_tile(qrows, qpos, g, k + (int64_t)p * L * d, v + (int64_t)p * L * d, L,
-                   d, block, scale, 0, lambda, tiles, starts, T,
+                   d, block, scale, 0, lambda, tiles, starts, T, sink_seed ? 0 : -1,
                    o + (int64_t)p * g * d, lse + (int64_t)p * g, st, mg);
         for (int t = 0; t < T; ++t) {
             if (tile_status)

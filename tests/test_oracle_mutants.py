@@ -29,6 +29,9 @@ MUTANTS = {
     "index_causal_off_by_one": [("> (int64_t)(i + 1) * q_block - 1)", "> (int64_t)(i + 1) * q_block)")],
     "mask_ignored": [("if (mask && !mask[((int64_t)mh * nq + i) * nk + j])", "if (0)")],
     "running_max_not_updated": [("if (mt > mprev[r])\n                mprev[r] = mt;", "(void)mt;")],
+    "reverse_ignored": [("        if (reverse)\n", "        if (0)\n")],
+    "seed_ignored": [("if (seed_tile >= 0 && tiles[t] != seed_tile)", "if (0)")],
+    "seed_from_split_first_tile": [("SCORE_TILE(seed_tile);", "SCORE_TILE(tiles[t]);")],
 }
 
 CHECKS = [
@@ -39,6 +42,8 @@ CHECKS = [
     pins.test_closed_form_keep,
     pins.test_closed_form_one_row_disagrees_keeps_tile,
     pins.test_closed_form_order_matters,
+    pins.test_closed_form_reverse_order,
+    pins.test_decode_sink_seed_closed_form,
     pins.test_decode_split_resets_running_max,
     pins.test_decode_gqa_group_vote,
     pins.test_index_matches_definition_and_causal,

@@ -204,6 +204,53 @@ def test_closed_form_order_matters():
     assert (r["status"][0, 0] == 2).all()
 
 
+def test_closed_form_reverse_order():
+    """Block-row reordering (the BLASST page's ablation, Figure 8): the tiles of
+    a row are visited in descending order.  With the big key in tile 1, tile 1
+    now sets the running max (10) and tile 0, whose max is 2, falls 8 below
+    it: skipped, and O = (e^10 v64 + sum_{k=65..127} v_k) / (e^10 + 63).  With
+    the big key in tile 0, reverse order keeps both tiles (tile 0's max is 8
+    above tile 1's)."""
+    q, k, v, v64 = _two_tile_case(2.0, swap=True)
+    r = oracle.prefill(q, k, v, 64, 1.0, False, math.exp(-5), reverse=True)
+    assert (r["status"][0, 0, :, 0] == 1).all() and (r["status"][0, 0, :, 1] == 2).all()
+    expect = (math.exp(10) * v64[64] + v64[65:].sum(0)) / (math.exp(10) + 63)
+    assert np.abs(r["o"][0, 0] - expect[None]).max() < 1e-12
+    assert np.abs(r["lse"][0, 0] - math.log(math.exp(10) + 63)).max() < 1e-12
+    np.testing.assert_allclose(r["margin"][0, 0, :, 0], -8.0 + 5.0, atol=1e-12)
+    q, k, v, _ = _two_tile_case(2.0)
+    r = oracle.prefill(q, k, v, 64, 1.0, False, math.exp(-5), reverse=True)
+    assert (r["status"][0, 0] == 2).all()
+
+
+def test_reverse_order_changes_nothing_without_skip():
+    """With lambda = 0 the visit order only changes the summation order: the
+    same visited tiles, every one executed, and the same O and LSE."""
+    q, k, v = inputs.blasst_prefill_qkv(1, 2, 1, 3 * 64 + 17, 64, "cpu", 11)
+    for causal in (False, True):
+        a = oracle.prefill(q, k, v, 64, 0.125, causal, 0.0)
+        b = oracle.prefill(q, k, v, 64, 0.125, causal, 0.0, reverse=True)
+        assert (a["status"] == b["status"]).all() and (a["status"] != 1).all()
+        assert np.abs(a["o"] - b["o"]).max() < 1e-12
+        assert np.abs(a["lse"] - b["lse"]).max() < 1e-12
+
+
+def test_reverse_order_with_mask_and_causal_first_tile_is_diagonal():
+    """Reverse order over a block mask: the first visited tile of every row is
+    its highest-index allowed tile, which is never skipped."""
+    rng = np.random.default_rng(5)
+    nb, block = 5, 64
+    N = nb * block - 9
+    m = (rng.random((1, nb, nb)) < 0.5).astype(np.uint8)
+    m[0, np.arange(nb), np.arange(nb)] = 1
+    q, k, v = inputs.blasst_prefill_qkv(1, 1, 1, N, 64, "cpu", 12)
+    r = oracle.prefill(q, k, v, block, 0.125, True, 0.5, mask=m, reverse=True)
+    for i in range(nb):
+        allowed = [j for j in range(nb) if m[0, i, j] and j <= i]
+        assert r["status"][0, 0, i, max(allowed)] == 2
+        assert set(np.nonzero(r["status"][0, 0, i])[0]) == set(allowed)
+
+
 def test_lambda_zero_and_one_edges():
     q, k, v, _ = _two_tile_case(2.0)
     r0 = oracle.prefill(q, k, v, 64, 1.0, False, 0.0)
@@ -285,6 +332,48 @@ def test_decode_split_resets_running_max():
     vv = np.concatenate([v[0, :64], v[0, 128:256]])
     p = np.exp(s - 20.0)
     assert np.abs(two["o"][0, 0] - (p @ vv) / p.sum()).max() < 1e-12
+
+
+def test_decode_sink_seed_closed_form():
+    """Sink seeding: every split after the first starts its running max from
+    key tile 0's row max.  Tile 0 holds a score of 10 (the sink), tiles 2 and 3
+    scores of 2.  Unseeded, split 2 restarts at -inf and executes both of its
+    tiles; seeded, both fall 8 below the sink (2 - 10 < -5) and are skipped,
+    leaving O = (e^10 v0 + sum_{k=1..63} v_k) / (e^10 + 63)."""
+    g, d, block = 1, 64, 64
+    L = 4 * block
+    q = np.zeros((1, g, d)); q[0, 0, 0] = 1.0
+    k = np.zeros((1, L, d)); k[0, 0, 0] = 10.0; k[0, 2 * block:, 0] = 2.0
+    v = np.random.default_rng(2).integers(-4, 5, (1, L, d)).astype(np.float64)
+    lam = math.exp(-5)
+    plain = oracle.decode(_bf16(q), _bf16(k), _bf16(v), block, 1.0, lam, 2)
+    assert list(plain["status"][0]) == [2, 1, 2, 2]
+    seeded = oracle.decode(_bf16(q), _bf16(k), _bf16(v), block, 1.0, lam, 2, sink_seed=True)
+    assert list(seeded["status"][0]) == [2, 1, 1, 1]
+    expect = (math.exp(10) * v[0, 0] + v[0, 1:64].sum(0)) / (math.exp(10) + 63)
+    assert np.abs(seeded["o"][0, 0] - expect).max() < 1e-12
+    np.testing.assert_allclose(seeded["margin"][0, 2:], [-3.0, -3.0], atol=1e-12)
+    # one split: seeding has nothing to seed
+    one_p = oracle.decode(_bf16(q), _bf16(k), _bf16(v), block, 1.0, lam, 1)
+    one_s = oracle.decode(_bf16(q), _bf16(k), _bf16(v), block, 1.0, lam, 1, sink_seed=True)
+    assert (one_p["status"] == one_s["status"]).all()
+    assert np.abs(one_p["o"] - one_s["o"]).max() == 0.0
+
+
+def test_decode_sink_seed_only_adds_skips():
+    """A seeded running max is never below the unseeded one, so seeding can
+    only turn executed tiles into skipped ones; with lambda = 0 it changes
+    nothing."""
+    q, k, v = inputs.blasst_decode_qkv(2, 8, 2, 40 * 64 + 5, 64, "cpu", 13)
+    qs, ks, vs = oracle.decode_problems(q, k, v, [(0, 0), (0, 1), (1, 0), (1, 1)])
+    a = oracle.decode(qs, ks, vs, 64, 0.125, 1e-2, 5)
+    b = oracle.decode(qs, ks, vs, 64, 0.125, 1e-2, 5, sink_seed=True)
+    assert ((b["status"] == 2) <= (a["status"] == 2)).all()
+    assert (b["status"] == 1).sum() > (a["status"] == 1).sum()
+    a0 = oracle.decode(qs, ks, vs, 64, 0.125, 0.0, 5)
+    b0 = oracle.decode(qs, ks, vs, 64, 0.125, 0.0, 5, sink_seed=True)
+    assert (a0["status"] == b0["status"]).all()
+    assert np.abs(a0["o"] - b0["o"]).max() == 0.0
 
 
 def test_decode_gqa_group_vote():
