@@ -157,7 +157,19 @@ int bsattn_fwd_prefill(const void* q, const void* k, const void* v, void* o, flo
                        float lambda, const int32_t* row_ptr, const int32_t* col_idx,
                        const int32_t* row_order, int mask_heads, uint8_t* tile_status,
                        int32_t* d_status, cudaStream_t stream) {
+  return bsattn_fwd_prefill_ex(q, k, v, o, lse, B, Hq, Hkv, N, d, block, scale, causal, lambda,
+                               row_ptr, col_idx, row_order, mask_heads, tile_status, 0u,
+                               d_status, stream);
+}
+
+int bsattn_fwd_prefill_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Hq, int Hkv, int N, int d, int block, float scale,
+                          int causal, float lambda, const int32_t* row_ptr,
+                          const int32_t* col_idx, const int32_t* row_order, int mask_heads,
+                          uint8_t* tile_status, unsigned flags, int32_t* d_status,
+                          cudaStream_t stream) {
   if (!q || !k || !v || !o) return BSATTN_ERR_INVALID_ARG;
+  if (flags & ~BSATTN_PREFILL_REVERSE) return BSATTN_ERR_INVALID_ARG;
   if (row_order && !row_ptr) return BSATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0) return BSATTN_ERR_INVALID_ARG;
   if (bad_lambda(lambda) || !std::isfinite(scale) || !(scale > 0.f)) return BSATTN_ERR_INVALID_ARG;
@@ -201,6 +213,7 @@ int bsattn_fwd_prefill(const void* q, const void* k, const void* v, void* o, flo
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
   p.use_skip = lambda > 0.f ? 1 : 0;
   p.thr_log2 = lambda > 0.f ? (float)std::log2((double)lambda) : -INFINITY;
+  p.reverse = (flags & BSATTN_PREFILL_REVERSE) ? 1 : 0;
   p.debug_stall = g_inject_stall;
   p.wait_limit_ns = g_wait_limit_ns;
   p.trace = g_trace;
@@ -236,8 +249,19 @@ int bsattn_fwd_decode(const void* q, const void* k, const void* v, void* o, floa
                       int Hq, int Hkv, int L, int d, int block, float scale, int causal,
                       float lambda, int num_splits, void* workspace, size_t workspace_bytes,
                       uint8_t* tile_status, int32_t* d_status, cudaStream_t stream) {
+  return bsattn_fwd_decode_ex(q, k, v, o, lse, B, Hq, Hkv, L, d, block, scale, causal, lambda,
+                              num_splits, workspace, workspace_bytes, tile_status, 0u, d_status,
+                              stream);
+}
+
+int bsattn_fwd_decode_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int Hq, int Hkv, int L, int d, int block, float scale, int causal,
+                         float lambda, int num_splits, void* workspace, size_t workspace_bytes,
+                         uint8_t* tile_status, unsigned flags, int32_t* d_status,
+                         cudaStream_t stream) {
   (void)causal;
   if (!q || !k || !v || !o || !workspace) return BSATTN_ERR_INVALID_ARG;
+  if (flags & ~BSATTN_DECODE_SINK_SEED) return BSATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0 || num_splits < 1)
     return BSATTN_ERR_INVALID_ARG;
   if (bad_lambda(lambda) || !std::isfinite(scale) || !(scale > 0.f)) return BSATTN_ERR_INVALID_ARG;
@@ -283,6 +307,7 @@ int bsattn_fwd_decode(const void* q, const void* k, const void* v, void* o, floa
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
   p.use_skip = lambda > 0.f ? 1 : 0;
   p.thr_log2 = lambda > 0.f ? (float)std::log2((double)lambda) : -INFINITY;
+  p.sink_seed = (flags & BSATTN_DECODE_SINK_SEED) ? 1 : 0;
   p.wait_limit_ns = g_wait_limit_ns;
   p.trace = g_trace;
   p.trace_n = g_trace_n;

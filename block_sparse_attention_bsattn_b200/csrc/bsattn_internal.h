@@ -34,6 +34,7 @@ struct PrefillParams {
   int use_skip;      // lambda > 0
   int debug_stall;   // test hook: the query tile is withheld from the tensor core
   int pair_tiles;    // two-slot kernel: consecutive query tiles of one head
+  int reverse;       // visit each row's key tiles in descending order
   unsigned long long wait_limit_ns;
   volatile int32_t* trace;  // debug: progress markers (host-visible memory) or null
   int trace_n;
@@ -50,6 +51,7 @@ struct DecodeParams {
   float scale_log2;
   float thr_log2;
   int use_skip;
+  int sink_seed;    // splits after the first start from key tile 0's row max
   unsigned long long wait_limit_ns;
   volatile int32_t* trace;
   int trace_n;

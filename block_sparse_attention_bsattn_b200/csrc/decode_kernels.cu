@@ -115,7 +115,11 @@ __global__ void __launch_bounds__(256, 1)
   const int b = bk / p.Hkv, kvh = bk % p.Hkv;
   const int t_begin = split * p.chunk;
   const int t_end = min(p.T, t_begin + p.chunk);
-  const int nt = max(0, t_end - t_begin);
+  // tile stream of the split: with sink seeding, step 0 scores key tile 0
+  // only to start the running max; step t >= sd is key tile t_begin + t - sd
+  const int sd = (p.sink_seed && split > 0 && t_end > t_begin) ? 1 : 0;
+  const int nt = max(0, t_end - t_begin) + sd;
+  auto tile_of = [&](int t) { return (sd && t == 0) ? 0 : t_begin + t - sd; };
   const int zc = b * p.Hkv + kvh;
 
   if (tid == 0) trace_mark(p.trace, p.trace_n, 16 + blockIdx.x, 1);
@@ -137,7 +141,7 @@ __global__ void __launch_bounds__(256, 1)
       mbar_arrive_expect_tx(&bars->k_full[s], C::T_BYTES);
       for (int hf = 0; hf < C::HALVES; ++hf)
         tma_load_3d(k_smem + s * C::T_BYTES + hf * C::T_HALF, &tmK, &bars->k_full[s], hf * 64,
-                    (t_begin + s) * BLK, zc);
+                    tile_of(s) * BLK, zc);
     }
   }
 
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(256, 1)
         for (int off = C::KPW; off < 32; off <<= 1)
 #pragma unroll
           for (int g = 0; g < G; ++g) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], off);
-        const int kpos = (t_begin + t) * BLK + key;
+        const int kpos = tile_of(t) * BLK + key;
         if (kpos >= p.L)
 #pragma unroll
           for (int g = 0; g < G; ++g) acc[g] = -INFINITY;
@@ -227,7 +231,7 @@ __global__ void __launch_bounds__(256, 1)
         mbar_arrive_expect_tx(&bars->k_full[ks], C::T_BYTES);
         for (int hf = 0; hf < C::HALVES; ++hf)
           tma_load_3d(k_smem + ks * C::T_BYTES + hf * C::T_HALF, &tmK, &bars->k_full[ks],
-                      hf * 64, (t_begin + tn) * BLK, zc);
+                      hf * 64, tile_of(tn) * BLK, zc);
       }
       issued_k = min(issued_k + 1, nt);
       // tile max per row (base-2 units), the vote, the running max
@@ -241,11 +245,13 @@ __global__ void __launch_bounds__(256, 1)
         mt[g] = m * p.scale_log2;
         all_pass = all_pass && (mt[g] - m_run[g] < p.thr_log2);
       }
-      const bool skip = p.use_skip && all_pass;
+      // the seed step only starts the running max: never kept, not a visit
+      const bool seed = sd && t == 0;
+      const bool skip = seed || (p.use_skip && all_pass);
 #pragma unroll
       for (int g = 0; g < G; ++g) m_run[g] = fmaxf(m_run[g], mt[g]);
-      if (tid == 0 && p.tile_status)
-        p.tile_status[(int64_t)zc * p.T + t_begin + t] = skip ? 1 : 2;
+      if (tid == 0 && p.tile_status && !seed)
+        p.tile_status[(int64_t)zc * p.T + tile_of(t)] = skip ? 1 : 2;
       if (!skip) {
         const int slot = kept_total % C::VST;
         // park the raw scores for the delayed P*V
@@ -256,7 +262,7 @@ __global__ void __launch_bounds__(256, 1)
           mbar_arrive_expect_tx(&bars->v_full[slot], C::T_BYTES);
           for (int hf = 0; hf < C::HALVES; ++hf)
             tma_load_3d(v_smem + slot * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[slot],
-                        hf * 64, (t_begin + t) * BLK, zc);
+                        hf * 64, tile_of(t) * BLK, zc);
         }
         ++issued_v;
         // lazy exponent shift

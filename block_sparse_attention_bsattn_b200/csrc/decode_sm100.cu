@@ -149,8 +149,10 @@ __global__ void __launch_bounds__(224, 1)
   const uint32_t tmem = bars->tmem_base;
   const uint64_t lim = p.wait_limit_ns;
 
-  // item n of this CTA -> (batch, kv head, split) and its tile range
-  auto item_of = [&](int n, int& b, int& kvh, int& split, int& t0, int& nt) {
+  // item n of this CTA -> (batch, kv head, split) and its tile stream: nt
+  // steps; with sink seeding (sd = 1) step 0 scores key tile 0 only to start
+  // the running max, and step t >= sd is key tile t0 + t - sd
+  auto item_of = [&](int n, int& b, int& kvh, int& split, int& t0, int& nt, int& sd) {
     const int it = blockIdx.x + n * gridDim.x;
     split = it % p.splits;
     const int bk = it / p.splits;
@@ -158,7 +160,10 @@ __global__ void __launch_bounds__(224, 1)
     kvh = bk % p.Hkv;
     t0 = split * p.chunk;
     nt = max(0, min(p.T, t0 + p.chunk) - t0);
+    sd = (p.sink_seed && split > 0 && nt > 0) ? 1 : 0;
+    nt += sd;
   };
+  auto tile_of = [](int t0, int sd, int t) { return (sd && t == 0) ? 0 : t0 + t - sd; };
   const int my_items = blockIdx.x < n_items ? (n_items - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
   if (warp == 0) {
@@ -169,8 +174,8 @@ __global__ void __launch_bounds__(224, 1)
       int g = 0;  // global tile counter
       bool ok = true;
       for (int n = 0; ok && n < my_items; ++n) {
-        int b, kvh, split, t0, nt;
-        item_of(n, b, kvh, split, t0, nt);
+        int b, kvh, split, t0, nt, sd;
+        item_of(n, b, kvh, split, t0, nt, sd);
         const int qs = n & 1;
         if (!mbar_wait(&bars->q_empty[qs], ((n >> 1) & 1) ^ 1, abort, lim)) break;
         mbar_arrive_expect_tx(&bars->q_full[qs], C::HALVES * C::Q_HALF);
@@ -183,7 +188,7 @@ __global__ void __launch_bounds__(224, 1)
           mbar_arrive_expect_tx(&bars->k_full[ks], C::T_BYTES);
           for (int hf = 0; hf < C::HALVES; ++hf)
             tma_load_3d(k_smem + ks * C::T_BYTES + hf * C::T_HALF, &tmK, &bars->k_full[ks],
-                        hf * 64, (t0 + t) * C::BLK, b * p.Hkv + kvh);
+                        hf * 64, tile_of(t0, sd, t) * C::BLK, b * p.Hkv + kvh);
         }
       }
       if (*abort) {
@@ -198,8 +203,8 @@ __global__ void __launch_bounds__(224, 1)
       int g = 0, kept = 0;
       bool ok = true;
       for (int n = 0; ok && n < my_items; ++n) {
-        int b, kvh, split, t0, nt;
-        item_of(n, b, kvh, split, t0, nt);
+        int b, kvh, split, t0, nt, sd;
+        item_of(n, b, kvh, split, t0, nt, sd);
         for (int t = 0; t < nt; ++t, ++g) {
           const int dq = g % C::DQ;
           if (!mbar_wait(&bars->dec_full[dq], (g / C::DQ) & 1, abort, lim)) { ok = false; break; }
@@ -211,7 +216,7 @@ __global__ void __launch_bounds__(224, 1)
           mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
           for (int hf = 0; hf < C::HALVES; ++hf)
             tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
-                        hf * 64, (t0 + t) * C::BLK, b * p.Hkv + kvh);
+                        hf * 64, tile_of(t0, sd, t) * C::BLK, b * p.Hkv + kvh);
           ++kept;
         }
       }
@@ -229,13 +234,13 @@ __global__ void __launch_bounds__(224, 1)
       const uint32_t q_addr = smem_u32(q_smem), p_addr = smem_u32(p_smem);
       // BMM1 stream state (runs up to LA tiles ahead of the BMM2 stream)
       int n1 = 0, t1 = 0, g1 = 0, nt1 = -1;
-      int b_, kvh_, split_, t0_;
+      int b_, kvh_, split_, t0_, sd_;
       bool ok = true;
       auto issue_next_bmm1 = [&]() -> int {  // 1 issued, 0 nothing left, -1 abort
         while (true) {
           if (nt1 < 0) {
             if (n1 >= my_items) return 0;
-            item_of(n1, b_, kvh_, split_, t0_, nt1);
+            item_of(n1, b_, kvh_, split_, t0_, nt1, sd_);
             t1 = 0;
             if (!mbar_wait(&bars->q_full[n1 & 1], (n1 >> 1) & 1, abort, lim)) return -1;
             tc_fence_after();
@@ -269,8 +274,8 @@ __global__ void __launch_bounds__(224, 1)
         if (issue_next_bmm1() < 0) ok = false;
       int g = 0, kept = 0;
       for (int n = 0; ok && n < my_items; ++n) {
-        int b, kvh, split, t0, nt;
-        item_of(n, b, kvh, split, t0, nt);
+        int b, kvh, split, t0, nt, sd;
+        item_of(n, b, kvh, split, t0, nt, sd);
         int kept_item = 0;
         for (int t = 0; t < nt; ++t, ++g) {
           if (issue_next_bmm1() < 0) { ok = false; break; }
@@ -309,8 +314,8 @@ __global__ void __launch_bounds__(224, 1)
     int g = 0, kept = 0;
     bool ok = true;
     for (int n = 0; ok && n < my_items; ++n) {
-      int b, kvh, split, t0, nt;
-      item_of(n, b, kvh, split, t0, nt);
+      int b, kvh, split, t0, nt, sd;
+      item_of(n, b, kvh, split, t0, nt, sd);
       float m_run[NC], m_ref[NC], lp[NC];
 #pragma unroll
       for (int c = 0; c < NC; ++c) { m_run[c] = -INFINITY; m_ref[c] = -INFINITY; lp[c] = 0.f; }
@@ -334,7 +339,9 @@ __global__ void __launch_bounds__(224, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
-        const bool key_ok = (t0 + t) * C::BLK + key < p.L;
+        const int jt = tile_of(t0, sd, t);
+        const bool seed = sd && t == 0;
+        const bool key_ok = jt * C::BLK + key < p.L;
         float s[NC];
 #pragma unroll
         for (int c = 0; c < NC; ++c) s[c] = (key_ok && c < G) ? __uint_as_float(r[c]) : -INFINITY;
@@ -375,7 +382,8 @@ __global__ void __launch_bounds__(224, 1)
           mt[c] = m * p.scale_log2;
           if (c < G) all_pass = all_pass && (mt[c] - m_run[c] < thr);
         }
-        const bool skip = p.use_skip && all_pass;
+        // the seed step only starts the running max: never kept, not a visit
+        const bool skip = seed || (p.use_skip && all_pass);
 #pragma unroll
         for (int c = 0; c < NC; ++c) m_run[c] = fmaxf(m_run[c], mt[c]);
         // the decision goes to the V producer and (for tile status) to memory
@@ -387,7 +395,8 @@ __global__ void __launch_bounds__(224, 1)
             bars->dec[dq] = skip ? 0 : 1;
             mbar_arrive(&bars->dec_full[dq]);
           }
-          if (p.tile_status) p.tile_status[(int64_t)(b * p.Hkv + kvh) * p.T + t0 + t] = skip ? 1 : 2;
+          if (p.tile_status && !seed)
+            p.tile_status[(int64_t)(b * p.Hkv + kvh) * p.T + jt] = skip ? 1 : 2;
         }
         if (__any_sync(0xffffffffu, *abort != 0)) { ok = false; break; }
         if (!skip) {

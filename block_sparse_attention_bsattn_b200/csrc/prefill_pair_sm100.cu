@@ -95,12 +95,16 @@ __global__ void __launch_bounds__(320, 1)
   int n;  // length of the shared K/V stream
   if (!p.pair_tiles) {
     const int PH = p.Hq / 2;
-    const int BP = p.B * PH;
     int i, bp;
     if (p.row_order) {
       bp = (int)(blockIdx.x / p.nq);
       i = p.row_order[(int)(blockIdx.x % p.nq)];
     } else if (p.causal) {
+      // longest query tile first across all head pairs.  (KV-head-major
+      // order brings DRAM reads down to the unique bytes but puts every SM
+      // on the same K/V lines at once, which measured slower: the L2-to-SM
+      // stream, not DRAM, paces this kernel.)
+      const int BP = p.B * PH;
       i = p.nq - 1 - (int)(blockIdx.x / BP);
       bp = (int)(blockIdx.x % BP);
     } else {
@@ -125,11 +129,10 @@ __global__ void __launch_bounds__(320, 1)
     ns[0] = ns[1] = n;
   } else {
     const int NP = (p.nq + 1) / 2;
-    const int BH = p.B * p.Hq;
     int m, bh;
-    if (p.causal) {                       // longest pairs first
-      m = NP - 1 - (int)(blockIdx.x / BH);
-      bh = (int)(blockIdx.x % BH);
+    if (p.causal) {  // head-major, longest pairs first: one head's K/V stays in L2
+      bh = (int)(blockIdx.x / NP);
+      m = NP - 1 - (int)(blockIdx.x % NP);
     } else {
       bh = (int)(blockIdx.x / NP);
       m = (int)(blockIdx.x % NP);
@@ -143,6 +146,20 @@ __global__ void __launch_bounds__(320, 1)
     n = max(ns[0], ns[1]);
   }
   const int kvh = hs[0] / (p.Hq / p.Hkv);
+  // stream step t -> key tile (ascending, or descending on request); slot e
+  // takes part in steps [tb[e], te[e]): a prefix of the stream in ascending
+  // order, a suffix in descending order
+  auto col_at = [&](int t) -> int {
+    const int u = p.reverse ? n - 1 - t : t;
+    return cols ? cols[u] : u;
+  };
+  int tb[2], te[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    tb[e] = p.reverse ? n - ns[e] : 0;
+    te[e] = p.reverse ? n : ns[e];
+  }
+
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -181,6 +198,7 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tensormap(&tmV);
       if (!p.debug_stall) {
         mbar_arrive_expect_tx(&bars->q_full, 2 * C::HALVES * BLK * 128);
+#pragma unroll
         for (int e = 0; e < 2; ++e)
           for (int hf = 0; hf < C::HALVES; ++hf)
             tma_load_3d(q_smem + e * C::Q_BYTES + hf * C::Q_HALF, &tmQ, &bars->q_full, hf * 64,
@@ -188,7 +206,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       int issued_k = 0, issued_v = 0;
       for (int t = 0; t < n; ++t) {
-        const int j = cols ? cols[t] : t;
+        const int j = col_at(t);
         const int ks = t % C::KST;
         if (!mbar_wait(&bars->k_empty[ks], ((t / C::KST) & 1) ^ 1, abort, lim)) break;
         mbar_arrive_expect_tx(&bars->k_full[ks], C::T_BYTES);
@@ -249,8 +267,8 @@ __global__ void __launch_bounds__(320, 1)
         ok = mbar_wait(&bars->k_full[0], 0, abort, lim);
         tc_fence_after();
         if (ok) {
-          if (ns[0] > 0) bmm1(0, 0);
-          if (ns[1] > 0) bmm1(1, 0);
+          if (tb[0] == 0 && te[0] > 0) bmm1(0, 0);
+          if (tb[1] == 0 && te[1] > 0) bmm1(1, 0);
           mma_commit(&bars->k_empty[0]);
         }
       }
@@ -262,20 +280,21 @@ __global__ void __launch_bounds__(320, 1)
         const bool more = t + 1 < n;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          if (t >= ns[e]) continue;  // this slot's visit list is shorter
-          if (!mbar_wait(&bars->p_ready[e], t & 1, abort, lim)) { ok = false; break; }
-          tc_fence_after();
-          const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[e]);
-          if (!skip) {
-            if (!v_ready) {
-              if (!mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) { ok = false; break; }
-              tc_fence_after();
-              v_ready = true;
+          if (t >= tb[e] && t < te[e]) {   // this slot takes part in step t
+            if (!mbar_wait(&bars->p_ready[e], (t - tb[e]) & 1, abort, lim)) { ok = false; break; }
+            tc_fence_after();
+            const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[e]);
+            if (!skip) {
+              if (!v_ready) {
+                if (!mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) { ok = false; break; }
+                tc_fence_after();
+                v_ready = true;
+              }
+              bmm2(e, t, kept[e] == 0);
+              ++kept[e];
             }
-            bmm2(e, t, kept[e] == 0);
-            ++kept[e];
           }
-          if (t + 1 < ns[e]) {
+          if (t + 1 >= tb[e] && t + 1 < te[e]) {
             if (!k_next) {   // first use of K_{t+1}
               const int ks = (t + 1) % C::KST;
               if (!mbar_wait(&bars->k_full[ks], ((t + 1) / C::KST) & 1, abort, lim)) { ok = false; break; }
@@ -304,18 +323,26 @@ __global__ void __launch_bounds__(320, 1)
     const int sw = (warp - 2) % 4;
     const int quarter = warp % 4;
     const int row = quarter * 32 + lane;
-    const int i = is[e];
+    // this slot's values as scalars (a runtime index would put the arrays in
+    // local memory)
+    const int i = e ? is[1] : is[0];
     const int r0 = i * BLK;
-    const int h = hs[e];
-    const int ne = ns[e];
+    const int h = e ? hs[1] : hs[0];
+    const int t_first = e ? tb[1] : tb[0];
+    const int ne = (e ? te[1] : te[0]) - t_first;
+    // key tile of this slot's t-th visit: u0 + du * t into the CSR row (or
+    // the tile index itself without one)
+    const int du = p.reverse ? -1 : 1;
+    const int u0 = p.reverse ? n - 1 - t_first : t_first;
     const bool valid = r0 + row < p.N;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t s_col = 256 * e, o_col = 256 * e + 128;
     float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
     int kept = 0;
     bool ok = true;
-    for (int t = 0; t < ne; ++t) {
-      const int j = cols ? cols[t] : t;
+    for (int t = 0; t < ne; ++t) {       // t counts this slot's tiles
+      const int u = u0 + du * t;
+      const int j = cols ? cols[u] : u;
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[e], t & 1, abort, lim))) {
         ok = false;
         break;

@@ -96,19 +96,18 @@ __global__ void __launch_bounds__(320, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // ---- work item.  With a row order (longest rows first, from the index
-  // builder) the items of one head run together, longest first; otherwise
-  // causal work runs in descending query-tile order (longest first) and
-  // non-causal work head by head.
-  const int BH = p.B * p.Hq;
+  // ---- work item: head by head (the heads of one KV head are adjacent, so
+  // the CTAs resident at one time share a K/V stream that stays in L2).
+  // Inside a head, a row order from the index builder (longest rows first),
+  // else causal work longest first, else ascending query tiles.
   int i, bh;
   if (p.row_order) {
     bh = (int)(blockIdx.x / p.nq);
     const int mh_o = p.mask_heads == 1 ? 0 : bh % p.Hq;
     i = p.row_order[(int64_t)mh_o * p.nq + (int)(blockIdx.x % p.nq)];
   } else if (p.causal) {
-    i = p.nq - 1 - (int)(blockIdx.x / BH);
-    bh = (int)(blockIdx.x % BH);
+    bh = (int)(blockIdx.x / p.nq);
+    i = p.nq - 1 - (int)(blockIdx.x % p.nq);
   } else {
     bh = (int)(blockIdx.x / p.nq);
     i = (int)(blockIdx.x % p.nq);
@@ -130,6 +129,11 @@ __global__ void __launch_bounds__(320, 1)
   } else {
     n = p.causal ? i + 1 : p.nk;
   }
+  // key tile of visit step t (ascending, or descending on request)
+  auto col_at = [&](int t) -> int {
+    const int u = p.reverse ? n - 1 - t : t;
+    return cols ? cols[u] : u;
+  };
 
   // debug trace: slot 16 + CTA = stage reached; CTA 0 also records per-role
   // progress, and an SM-clock timeline of its first tiles from slot 1024 on
@@ -184,7 +188,7 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tensormap(&tmV);
       int issued_k = 0, issued_v = 0;
       for (int t = 0; t < n; ++t) {
-        const int j = cols ? cols[t] : t;
+        const int j = col_at(t);
         const int ks = t % C::KST;
         if (!mbar_wait(&bars->k_empty[ks], ((t / C::KST) & 1) ^ 1, abort, lim)) break;
         mbar_arrive_expect_tx(&bars->k_full[ks], C::T_BYTES);
@@ -313,7 +317,7 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) mbar_arrive(&bars->q_ready);
     }
     for (int t = 0; t < n; ++t) {
-      const int j = cols ? cols[t] : t;
+      const int j = col_at(t);
       const int sb = t & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (t >> 1) & 1, abort, lim))) {
         ok = false;

@@ -42,18 +42,29 @@ _lib.bsattn_build_index.restype = _I
 _lib.bsattn_fwd_prefill.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F,
                                     _P, _P, _P, _I, _P, _P, _P]
 _lib.bsattn_fwd_prefill.restype = _I
+_lib.bsattn_fwd_prefill_ex.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F,
+                                       _P, _P, _P, _I, _P, ctypes.c_uint, _P, _P]
+_lib.bsattn_fwd_prefill_ex.restype = _I
 _lib.bsattn_decode_workspace_size.argtypes = [_I, _I, _I, _I]
 _lib.bsattn_decode_workspace_size.restype = _SZ
 _lib.bsattn_fwd_decode.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F, _I,
                                    _P, _SZ, _P, _P, _P]
 _lib.bsattn_fwd_decode.restype = _I
+_lib.bsattn_fwd_decode_ex.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F,
+                                      _I, _P, _SZ, _P, ctypes.c_uint, _P, _P]
+_lib.bsattn_fwd_decode_ex.restype = _I
 _lib.bsattn_fwd_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I,
                                            _F, _I, _P, _P, _P]
 _lib.bsattn_fwd_decode_noalloc.restype = _I
 
+# option bits of the _ex entry points (include/bsattn.h)
+PREFILL_REVERSE = 0x1
+DECODE_SINK_SEED = 0x1
+
 EXPORTED = ("bsattn_status_string", "bsattn_version", "bsattn_debug_set", "bsattn_debug_trace",
             "bsattn_build_index",
-            "bsattn_fwd_prefill", "bsattn_decode_workspace_size", "bsattn_fwd_decode",
+            "bsattn_fwd_prefill", "bsattn_fwd_prefill_ex", "bsattn_decode_workspace_size",
+            "bsattn_fwd_decode", "bsattn_fwd_decode_ex",
             "bsattn_fwd_decode_noalloc")
 
 
@@ -140,8 +151,11 @@ def bsattn_fwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
                        o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                        want_lse: bool = True, tile_status: Optional[torch.Tensor] = None,
                        status: Optional[torch.Tensor] = None,
-                       row_order: Optional[torch.Tensor] = None, stream=None):
-    """q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 -> (o [B,Hq,N,d] bf16, lse [B,Hq,N] fp32 or None)."""
+                       row_order: Optional[torch.Tensor] = None, stream=None,
+                       reverse: bool = False):
+    """q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 -> (o [B,Hq,N,d] bf16, lse [B,Hq,N] fp32 or None).
+    reverse: visit each row's key tiles in descending order (calls
+    bsattn_fwd_prefill_ex with BSATTN_PREFILL_REVERSE)."""
     _check(q, "q", torch.bfloat16, 4)
     _check(k, "k", torch.bfloat16, 4)
     _check(v, "v", torch.bfloat16, 4)
@@ -155,10 +169,14 @@ def bsattn_fwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
         o = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
-    rc = _lib.bsattn_fwd_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
-                                 int(block), float(scale), int(causal), float(lam), _ptr(row_ptr),
-                                 _ptr(col_idx), _ptr(row_order), int(mask_heads),
-                                 _ptr(tile_status), _ptr(status), _stream(stream))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, int(block),
+            float(scale), int(causal), float(lam), _ptr(row_ptr), _ptr(col_idx), _ptr(row_order),
+            int(mask_heads), _ptr(tile_status))
+    flags = PREFILL_REVERSE if reverse else 0
+    if flags:
+        rc = _lib.bsattn_fwd_prefill_ex(*args, flags, _ptr(status), _stream(stream))
+    else:
+        rc = _lib.bsattn_fwd_prefill(*args, _ptr(status), _stream(stream))
     if rc:
         raise BsattnError(rc, "bsattn_fwd_prefill")
     return o, lse
@@ -173,8 +191,11 @@ def bsattn_fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: 
                       o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                       want_lse: bool = True, workspace: Optional[torch.Tensor] = None,
                       tile_status: Optional[torch.Tensor] = None,
-                      status: Optional[torch.Tensor] = None, stream=None):
-    """q [B,Hq,d], k/v [B,Hkv,L,d] bf16 -> (o [B,Hq,d] bf16, lse [B,Hq] fp32 or None)."""
+                      status: Optional[torch.Tensor] = None, stream=None,
+                      sink_seed: bool = False):
+    """q [B,Hq,d], k/v [B,Hkv,L,d] bf16 -> (o [B,Hq,d] bf16, lse [B,Hq] fp32 or None).
+    sink_seed: splits after the first start their running max from key tile
+    0's row max (calls bsattn_fwd_decode_ex with BSATTN_DECODE_SINK_SEED)."""
     _check(q, "q", torch.bfloat16, 3)
     _check(k, "k", torch.bfloat16, 4)
     _check(v, "v", torch.bfloat16, 4)
@@ -191,10 +212,13 @@ def bsattn_fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: 
     need = bsattn_decode_workspace_size(B, Hq, d, num_splits)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    rc = _lib.bsattn_fwd_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, L, d,
-                                int(block), float(scale), 0, float(lam), int(num_splits),
-                                _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                _ptr(tile_status), _ptr(status), _stream(stream))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, L, d, int(block),
+            float(scale), 0, float(lam), int(num_splits), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _ptr(tile_status))
+    if sink_seed:
+        rc = _lib.bsattn_fwd_decode_ex(*args, DECODE_SINK_SEED, _ptr(status), _stream(stream))
+    else:
+        rc = _lib.bsattn_fwd_decode(*args, _ptr(status), _stream(stream))
     if rc:
         raise BsattnError(rc, "bsattn_fwd_decode")
     return o, lse

@@ -145,6 +145,29 @@ int bsattn_fwd_prefill(const void *q, const void *k, const void *v, void *o, flo
                        const int32_t *row_order, int mask_heads, uint8_t *tile_status,
                        int32_t *d_status, cudaStream_t stream);
 
+/* Option bits of bsattn_fwd_prefill_ex. */
+#define BSATTN_PREFILL_REVERSE 0x1u
+
+/*
+ * bsattn_fwd_prefill_ex -- bsattn_fwd_prefill with option bits; flags = 0 is
+ * exactly bsattn_fwd_prefill.  Unknown bits give BSATTN_ERR_INVALID_ARG.
+ *
+ * BSATTN_PREFILL_REVERSE: every query tile visits its key tiles in descending
+ * order instead of ascending.  This is the block-row reordering of "BLASST:
+ * Dynamic Blocked Attention Sparsity via Softmax Thresholding" (ablation
+ * study, Figure 8): the tiles nearest the query (the local window, which
+ * usually holds the largest scores) then set the running max first, and the
+ * farther tiles are tested against it.  The skip decisions -- and so O, LSE
+ * and tile_status -- are those of the reversed order; with lambda = 0 only
+ * the summation order changes.
+ */
+int bsattn_fwd_prefill_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                          int B, int Hq, int Hkv, int N, int d, int block, float scale,
+                          int causal, float lambda, const int32_t *row_ptr,
+                          const int32_t *col_idx, const int32_t *row_order, int mask_heads,
+                          uint8_t *tile_status, unsigned flags, int32_t *d_status,
+                          cudaStream_t stream);
+
 /*
  * bsattn_decode_workspace_size -- bytes of scratch bsattn_fwd_decode needs:
  * per (batch, query head, split) d fp32 partial outputs plus the split's
@@ -179,6 +202,29 @@ int bsattn_fwd_decode(const void *q, const void *k, const void *v, void *o, floa
                       int Hq, int Hkv, int L, int d, int block, float scale, int causal,
                       float lambda, int num_splits, void *workspace, size_t workspace_bytes,
                       uint8_t *tile_status, int32_t *d_status, cudaStream_t stream);
+
+/* Option bits of bsattn_fwd_decode_ex. */
+#define BSATTN_DECODE_SINK_SEED 0x1u
+
+/*
+ * bsattn_fwd_decode_ex -- bsattn_fwd_decode with option bits; flags = 0 is
+ * exactly bsattn_fwd_decode.  Unknown bits give BSATTN_ERR_INVALID_ARG.
+ *
+ * BSATTN_DECODE_SINK_SEED: every split but the first starts its running max
+ * from the row max of key tile 0 -- the tile that holds the attention sink --
+ * instead of -inf.  The split scores tile 0 for this (one more K tile read per
+ * split) without visiting or executing it; tile_status and the result count
+ * tile 0 only in the first split.  A later split can then skip tiles that the
+ * sink dominates, where a split starting at -inf must execute its first tile
+ * and test the rest against its own, smaller maxima.  (The pages define no
+ * split-KV; this variant keeps their skip rule and only changes the starting
+ * value of each split's running max.)
+ */
+int bsattn_fwd_decode_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                         int B, int Hq, int Hkv, int L, int d, int block, float scale, int causal,
+                         float lambda, int num_splits, void *workspace, size_t workspace_bytes,
+                         uint8_t *tile_status, unsigned flags, int32_t *d_status,
+                         cudaStream_t stream);
 
 /*
  * bsattn_fwd_decode_noalloc -- bsattn_fwd_decode for callers that cannot

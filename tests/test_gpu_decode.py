@@ -18,7 +18,7 @@ def _ops():
     return ops
 
 
-def _run(q, k, v, block, splits, scale, lam):
+def _run(q, k, v, block, splits, scale, lam, sink_seed=False):
     ops = _ops()
     B, Hq, d = q.shape
     Hkv, L = k.shape[1], k.shape[2]
@@ -26,21 +26,22 @@ def _run(q, k, v, block, splits, scale, lam):
     st = torch.zeros(B, Hkv, T, dtype=torch.uint8, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     o, lse = ops.bsattn_fwd_decode(q.cuda(), k.cuda(), v.cuda(), block, splits, scale, lam,
-                                   tile_status=st, status=status)
+                                   tile_status=st, status=status, sink_seed=sink_seed)
     torch.cuda.synchronize()
     assert status.item() == 0, ops.bsattn_status_string(status.item())
     return o, lse, st
 
 
-def _check(q, k, v, block, splits, scale, lam, pairs=None, what=""):
-    o, lse, st = _run(q, k, v, block, splits, scale, lam)
+def _check(q, k, v, block, splits, scale, lam, pairs=None, what="", sink_seed=False):
+    o, lse, st = _run(q, k, v, block, splits, scale, lam, sink_seed)
     B, Hq, d = q.shape
     Hkv = k.shape[1]
     g = Hq // Hkv
     if pairs is None:
         pairs = [(b, h) for b in range(B) for h in range(Hkv)]
     qs, ks, vs = oracle.decode_problems(q, k, v, pairs)
-    ref = oracle.decode(qs.cpu(), ks.cpu(), vs.cpu(), block, scale, lam, splits)
+    ref = oracle.decode(qs.cpu(), ks.cpu(), vs.cpu(), block, scale, lam, splits,
+                        sink_seed=sink_seed)
     o_c, lse_c, st_c = o.float().cpu().numpy(), lse.cpu().numpy(), st.cpu().numpy()
     for p, (b, kvh) in enumerate(pairs):
         compare_outputs(o_c[b, kvh * g:(kvh + 1) * g], ref["o"][p], lse_c[b, kvh * g:(kvh + 1) * g],
@@ -72,6 +73,26 @@ def test_decode_table4_shape_shrunk(a):
     with fewer sequences and a shorter cache."""
     q, k, v = inputs.blasst_decode_qkv(3, 32, 4, 8192, 128, "cpu", 4243)
     _check(q, k, v, 128, 16, 1 / math.sqrt(128), inputs.lambda_for(a, 8192), what=f"t4 a={a}")
+
+
+@pytest.mark.parametrize("d,block,g", [(128, 128, 4), (128, 128, 8), (64, 128, 3),
+                                       (128, 64, 4), (64, 64, 1)])
+def test_sink_seeded_splits(d, block, g):
+    """Splits after the first start their running max from key tile 0's row
+    max: both decode kernels against the oracle's seeded splits, and more V
+    tiles skipped than without seeding."""
+    B, Hkv, L = 2, 2, 23 * block + 7
+    q, k, v = inputs.blasst_decode_qkv(B, Hkv * g, Hkv, L, d, "cpu", 57 + g + block)
+    lam = inputs.lambda_for(10.0, L)
+    seeded = _check(q, k, v, block, 5, 1 / math.sqrt(d), lam, what=f"seed d{d} b{block} g{g}",
+                    sink_seed=True)
+    plain = _check(q, k, v, block, 5, 1 / math.sqrt(d), lam, what="plain")
+    assert (seeded["status"] == 1).sum() > (plain["status"] == 1).sum()
+
+
+def test_sink_seed_with_empty_splits():
+    q, k, v = inputs.blasst_decode_qkv(1, 4, 1, 300, 128, "cpu", 9)
+    _check(q, k, v, 128, 8, 1 / math.sqrt(128), 1e-2, what="seeded empty splits", sink_seed=True)
 
 
 def test_more_splits_than_tiles():

@@ -18,7 +18,7 @@ def _ops():
     return ops
 
 
-def _run_gpu(w, lam, mask=None, mask_heads=1, ordered=True):
+def _run_gpu(w, lam, mask=None, mask_heads=1, ordered=True, reverse=False):
     """Index (with the longest-first row order unless `ordered` is False) and
     prefill through the C ABI; returns (o, lse, tile_status)."""
     ops = _ops()
@@ -33,15 +33,17 @@ def _run_gpu(w, lam, mask=None, mask_heads=1, ordered=True):
     st = torch.zeros(w.B, w.Hq, w.nq, w.nk, dtype=torch.uint8, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     o, lse = ops.bsattn_fwd_prefill(q, k, v, w.block, w.scale, w.causal, lam, rp, ci, mask_heads,
-                                    tile_status=st, status=status, row_order=order)
+                                    tile_status=st, status=status, row_order=order,
+                                    reverse=reverse)
     torch.cuda.synchronize()
     assert status.item() == 0, ops.bsattn_status_string(status.item())
     return o, lse, st
 
 
-def _check(w, lam, mask=None, what="", ordered=True):
-    o, lse, st = _run_gpu(w, lam, mask, ordered=ordered)
-    ref = oracle.prefill(w.q, w.k, w.v, w.block, w.scale, w.causal, lam, mask=mask)
+def _check(w, lam, mask=None, what="", ordered=True, reverse=False):
+    o, lse, st = _run_gpu(w, lam, mask, ordered=ordered, reverse=reverse)
+    ref = oracle.prefill(w.q, w.k, w.v, w.block, w.scale, w.causal, lam, mask=mask,
+                         reverse=reverse)
     compare_outputs(o, ref["o"], lse, ref["lse"], what)
     compare_status(st, ref["status"], ref["margin"], what)
     return ref
@@ -114,6 +116,51 @@ def test_blasst_prefill_one_head_per_kv_head(a):
     w = inputs.Workload("t4", B, H, H, N, 128, 128, True, "prefill", 1 / math.sqrt(128), None,
                         q=q, k=k, v=v)
     _check(w, inputs.lambda_for(a, N), None, f"table4-shape a={a}")
+
+
+@pytest.mark.parametrize("hq,hkv,block,causal", [
+    (4, 2, 128, True),     # two heads of one KV head per CTA
+    (1, 1, 128, True),     # two consecutive query tiles per CTA, odd count
+    (3, 1, 128, False),    # two consecutive query tiles, non-causal
+    (2, 1, 64, True),      # one query tile per CTA
+])
+def test_reverse_visit_order(hq, hkv, block, causal):
+    """Block-row reordering: every query tile visits its key tiles in
+    descending order; decisions, O, LSE and tile status match the oracle's
+    reversed visit.  Inputs: the first key of tile j scores 3 (j + 1) against
+    every query and the rest score near 0, so the descending visit meets the
+    largest score first and skips the earlier tiles (ln 0.1 > -3), while the
+    ascending visit keeps every tile."""
+    N = 5 * block + 21
+    g = torch.Generator().manual_seed(21 + block)
+    q = 0.1 * torch.randn(2, hq, N, 128, generator=g)
+    q[..., 0] = 1.0
+    k = 0.1 * torch.randn(2, hkv, N, 128, generator=g)
+    for j in range(-(-N // block)):
+        k[:, :, j * block, 0] = 3.0 * (j + 1)
+    v = torch.randn(2, hkv, N, 128, generator=g)
+    q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
+    w = inputs.Workload("rev", 2, hq, hkv, N, 128, block, causal, "prefill", 1.0, None,
+                        q=q, k=k, v=v)
+    ref = _check(w, 0.1, None, f"reverse h{hq}/{hkv} b{block} c{causal}", reverse=True)
+    assert (ref["status"] == 1).sum() > 0
+    ref = _check(w, 0.1, None, f"ascending h{hq}/{hkv} b{block} c{causal}")
+    assert (ref["status"] == 1).sum() == 0
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_reverse_visit_order_with_masks(block):
+    """Reverse order over per-head and shared block masks (CSR visit lists)."""
+    rng = np.random.default_rng(block)
+    N = 6 * block - 3
+    nb = -(-N // block)
+    q, k, v = inputs.blasst_prefill_qkv(1, 4, 2, N, 64, "cpu", 8)
+    w = inputs.Workload("revm", 1, 4, 2, N, 64, block, True, "prefill", 0.125, None,
+                        q=q, k=k, v=v)
+    for heads in (1, 4):
+        m = (rng.random((heads, nb, nb)) < 0.6).astype(np.uint8)
+        m[:, np.arange(nb), np.arange(nb)] = 1
+        _check(w, 0.02, m, f"reverse mask{heads}", reverse=True)
 
 
 def test_short_sequence_single_partial_tile():
