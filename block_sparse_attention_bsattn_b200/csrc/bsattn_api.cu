@@ -169,7 +169,7 @@ int bsattn_fwd_prefill_ex(const void* q, const void* k, const void* v, void* o, 
                           uint8_t* tile_status, unsigned flags, int32_t* d_status,
                           cudaStream_t stream) {
   if (!q || !k || !v || !o) return BSATTN_ERR_INVALID_ARG;
-  if (flags & ~BSATTN_PREFILL_REVERSE) return BSATTN_ERR_INVALID_ARG;
+  if (flags & ~(BSATTN_PREFILL_REVERSE | BSATTN_PREFILL_SKIP_V)) return BSATTN_ERR_INVALID_ARG;
   if (row_order && !row_ptr) return BSATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0) return BSATTN_ERR_INVALID_ARG;
   if (bad_lambda(lambda) || !std::isfinite(scale) || !(scale > 0.f)) return BSATTN_ERR_INVALID_ARG;
@@ -214,6 +214,7 @@ int bsattn_fwd_prefill_ex(const void* q, const void* k, const void* v, void* o, 
   p.use_skip = lambda > 0.f ? 1 : 0;
   p.thr_log2 = lambda > 0.f ? (float)std::log2((double)lambda) : -INFINITY;
   p.reverse = (flags & BSATTN_PREFILL_REVERSE) ? 1 : 0;
+  p.skip_v = (flags & BSATTN_PREFILL_SKIP_V) ? 1 : 0;
   p.debug_stall = g_inject_stall;
   p.wait_limit_ns = g_wait_limit_ns;
   p.trace = g_trace;

@@ -35,6 +35,7 @@ struct PrefillParams {
   int debug_stall;   // test hook: the query tile is withheld from the tensor core
   int pair_tiles;    // two-slot kernel: consecutive query tiles of one head
   int reverse;       // visit each row's key tiles in descending order
+  int skip_v;        // load V only for tiles some query tile keeps
   unsigned long long wait_limit_ns;
   volatile int32_t* trace;  // debug: progress markers (host-visible memory) or null
   int trace_n;

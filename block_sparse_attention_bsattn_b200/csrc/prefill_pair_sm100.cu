@@ -13,9 +13,15 @@
 // tiles P = exp(S - m), the row sums and O += P V.  The two heads' skip
 // decisions are independent.
 //
-// 10 warps:
+// 10 warps (11 with V skipping):
 //   warp 0      TMA producer: Q of both heads, then K_j (3-stage ring) and V_j
 //               (2-stage ring)
+//   warp 10     with V skipping only: the V producer.  The section on the
+//               prefill kernel keeps every V load (the decision comes too late
+//               to hide a conditional load's latency); as an option, a slot's
+//               softmax sends each decision through a queue and V_j is loaded
+//               only when some slot keeps tile j, which halves the bytes a
+//               skipped step pulls from L2.
 //   warp 1      TMEM owner, MMA issuer.  The two query tiles ping-pong: after
 //               head A's P is ready its BMM2 and its next BMM1 are issued, then
 //               head B's, so the tensor core works on one head while the other
@@ -52,8 +58,8 @@ struct PairCfg {
   static constexpr int BAR_OFF = V_OFF + VST * T_BYTES;
   static constexpr int SMEM = BAR_OFF + 512 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 320;
   static constexpr float TAU = 8.0f;
+  static constexpr int DQ = 4;                          // decision queue (V skipping)
 };
 
 struct PairBarriers {
@@ -64,15 +70,17 @@ struct PairBarriers {
   uint64_t p_ready[2];      // per head
   uint64_t o_done[2];       // per head
   uint64_t vote_bar[2][2];  // per head, tile parity
+  uint64_t dq_full[2][4], dq_empty[2][4];   // per slot: decisions to the V producer
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
   int skip_flag[2];
   int vote[2][2][4];        // head, tile parity, warp
+  int dval[2][4];           // 1 = kept
 };
 
-template <int D>
-__global__ void __launch_bounds__(320, 1)
+template <int D, bool SKIPV>
+__global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -175,6 +183,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&bars->o_done[s], 1);
       mbar_init(&bars->vote_bar[s][0], 4);
       mbar_init(&bars->vote_bar[s][1], 4);
+      for (int x = 0; x < C::DQ; ++x) {
+        mbar_init(&bars->dq_full[s][x], 1);
+        mbar_init(&bars->dq_empty[s][x], 1);
+      }
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -214,6 +226,7 @@ __global__ void __launch_bounds__(320, 1)
           tma_load_3d(k_smem + ks * C::T_BYTES + hf * C::T_HALF, &tmK, &bars->k_full[ks],
                       hf * 64, j * BLK, b * p.Hkv + kvh);
         ++issued_k;
+        if (SKIPV) continue;   // warp 10 loads V
         const int vs = t % C::VST;
         if (!mbar_wait(&bars->v_empty[vs], ((t / C::VST) & 1) ^ 1, abort, lim)) break;
         mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
@@ -229,6 +242,39 @@ __global__ void __launch_bounds__(320, 1)
           mbar_wait_drain(&bars->v_full[t % C::VST], (t / C::VST) & 1, lim);
         if (!p.debug_stall) mbar_wait_drain(&bars->q_full, 0, lim);
       }
+    }
+  } else if (SKIPV && warp == 10) {
+    // ======================================================== V producer (V skipping)
+    if (lane == 0 && n > 0) {
+      prefetch_tensormap(&tmV);
+      int vc = 0;   // V tiles loaded
+      bool ok = true;
+      for (int t = 0; ok && t < n; ++t) {
+        bool need = false;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          if (t < tb[e] || t >= te[e]) continue;
+          const int tl = t - tb[e];
+          if (!mbar_wait(&bars->dq_full[e][tl % C::DQ], (tl / C::DQ) & 1, abort, lim)) {
+            ok = false;
+            break;
+          }
+          need = need || *reinterpret_cast<volatile int*>(&bars->dval[e][tl % C::DQ]) != 0;
+          mbar_arrive(&bars->dq_empty[e][tl % C::DQ]);
+        }
+        if (!ok || !need) continue;
+        const int vs = vc % C::VST;
+        if (!mbar_wait(&bars->v_empty[vs], ((vc / C::VST) & 1) ^ 1, abort, lim)) break;
+        mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
+        const int j = col_at(t);
+        for (int hf = 0; hf < C::HALVES; ++hf)
+          tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
+                      hf * 64, j * BLK, b * p.Hkv + kvh);
+        ++vc;
+      }
+      if (*abort)
+        for (int x = (vc > C::VST ? vc - C::VST : 0); x < vc; ++x)
+          mbar_wait_drain(&bars->v_full[x % C::VST], (x / C::VST) & 1, lim);
     }
   } else if (warp == 1) {
     // ======================================================== MMA issuer
@@ -252,9 +298,8 @@ __global__ void __launch_bounds__(320, 1)
         }
         mma_commit(&bars->s_full[e]);
       };
-      // O_e += P_e V_t, P_e in TMEM over S_e
-      auto bmm2 = [&](int e, int t, int first) {
-        const int vs = t % C::VST;
+      // O_e += P_e V, P_e in TMEM over S_e, V in ring slot vs
+      auto bmm2 = [&](int e, int vs, int first) {
 #pragma unroll
         for (int kk = 0; kk < BLK / 16; ++kk) {
           const uint32_t bb = v_addr + vs * C::T_BYTES + kk * (16 * 128);
@@ -273,8 +318,10 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       int kept[2] = {0, 0};
+      int vc = 0;   // V tiles loaded so far (V skipping: only the kept steps')
       for (int t = 0; ok && t < n; ++t) {
-        const int vs = t % C::VST;
+        const int vi = SKIPV ? vc : t;
+        const int vs = vi % C::VST;
         bool v_ready = false;
         bool k_next = false;        // K_{t+1} waited for
         const bool more = t + 1 < n;
@@ -286,11 +333,11 @@ __global__ void __launch_bounds__(320, 1)
             const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[e]);
             if (!skip) {
               if (!v_ready) {
-                if (!mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) { ok = false; break; }
+                if (!mbar_wait(&bars->v_full[vs], (vi / C::VST) & 1, abort, lim)) { ok = false; break; }
                 tc_fence_after();
                 v_ready = true;
               }
-              bmm2(e, t, kept[e] == 0);
+              bmm2(e, vs, kept[e] == 0);
               ++kept[e];
             }
           }
@@ -306,12 +353,14 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (!ok) break;
         if (more) mma_commit(&bars->k_empty[(t + 1) % C::KST]);
-        // release V_t: consumed (or not needed) by both heads
-        if (!v_ready) {
+        // release V_t: consumed (or not needed) by both heads; with V skipping
+        // a step that no slot keeps has no V tile
+        if (v_ready) {
+          mma_commit(&bars->v_empty[vs]);
+          ++vc;
+        } else if (!SKIPV) {
           if (!mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) break;
           mbar_arrive(&bars->v_empty[vs]);
-        } else {
-          mma_commit(&bars->v_empty[vs]);
         }
       }
       mma_commit(&bars->drain);
@@ -388,6 +437,19 @@ __global__ void __launch_bounds__(320, 1)
         }
         volatile int* vv = bars->vote[e][t & 1];
         skip = vv[0] & vv[1] & vv[2] & vv[3];
+      }
+      if (SKIPV) {   // the decision to the V producer, before any exponential
+        if (sw == 0 && lane == 0) {
+          const int dq = t % C::DQ;
+          if (mbar_wait(&bars->dq_empty[e][dq], ((t / C::DQ) & 1) ^ 1, abort, lim)) {
+            bars->dval[e][dq] = skip ? 0 : 1;
+            mbar_arrive(&bars->dq_full[e][dq]);
+          }
+        }
+        if (__any_sync(0xffffffffu, *abort != 0)) {
+          ok = false;
+          break;
+        }
       }
       m_run = fmaxf(m_run, mt);
       if (sw == 0 && lane == 0 && p.tile_status && (unsigned)j < (unsigned)p.nk)
@@ -493,17 +555,25 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
+template <int D, bool SKIPV>
+static cudaError_t launch_pair(const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const PrefillParams& p, int grid,
+                               cudaStream_t stream) {
+  using C = PairCfg<D>;
+  static_assert(C::SMEM <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(prefill_pair_kernel<D, SKIPV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  prefill_pair_kernel<D, SKIPV><<<grid, SKIPV ? 352 : 320, C::SMEM, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_prefill_pair(const CUtensorMap& tq, const CUtensorMap& tk,
                                 const CUtensorMap& tv, const PrefillParams& p, int grid,
                                 cudaStream_t stream) {
-  using C = PairCfg<D>;
-  static_assert(C::SMEM <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(prefill_pair_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return e;
-  prefill_pair_kernel<D><<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  return p.skip_v ? launch_pair<D, true>(tq, tk, tv, p, grid, stream)
+                  : launch_pair<D, false>(tq, tk, tv, p, grid, stream);
 }
 
 template cudaError_t launch_prefill_pair<128>(const CUtensorMap&, const CUtensorMap&,

@@ -54,14 +54,14 @@ struct PrefillCfg {
   static constexpr int BAR_OFF = XM_OFF + 6 * 128 * 4;
   // + alignment slack; at least 116 KB so that one CTA (which holds all 512
   // TMEM columns) is resident per SM
-  static constexpr int SMEM_USED = BAR_OFF + 256 + 1024;
+  static constexpr int SMEM_USED = BAR_OFF + 512 + 1024;
   static constexpr int SMEM = SMEM_USED > 118784 ? SMEM_USED : 118784;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0;             // S[b] at b * 128
   static constexpr uint32_t O_COL = 256;
   static constexpr uint32_t Q_COL = 384;           // Q tile, bf16 pairs (d/2 columns)
-  static constexpr int THREADS = 320;
   static constexpr float TAU = 8.0f;               // lazy-rescale slack (base-2 units)
+  static constexpr int DQ = 4;                     // decision queue (V skipping)
 };
 
 struct PrefillBarriers {
@@ -75,17 +75,22 @@ struct PrefillBarriers {
   uint64_t vote_bar[2];
   uint64_t epi_bar;
   uint32_t tmem_base;
+  uint64_t dq_full[4], dq_empty[4];   // decisions to the V producer (V skipping)
   int abort;
   int skip_flag[2];
   int vote[2][8];
+  int dval[4];           // 1 = kept
 };
 
-template <int D, int BLK>
-__global__ void __launch_bounds__(320, 1)
+// SKIPV: V tiles are loaded only for executed tiles, by an eleventh warp that
+// reads each tile's decision from a queue (the page's prefill kernel loads
+// every V tile; this is the option it names for memory-bound cases).
+template <int D, int BLK, bool SKIPV>
+__global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   using C = PrefillCfg<D, BLK>;
-  static_assert(sizeof(PrefillBarriers) <= 256, "barrier block");
+  static_assert(sizeof(PrefillBarriers) <= 512, "barrier block");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -165,6 +170,10 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->vote_bar[0], 8);
     mbar_init(&bars->vote_bar[1], 8);
+    for (int x = 0; x < C::DQ; ++x) {
+      mbar_init(&bars->dq_full[x], 1);
+      mbar_init(&bars->dq_empty[x], 1);
+    }
     mbar_init(&bars->epi_bar, 8);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -196,6 +205,7 @@ __global__ void __launch_bounds__(320, 1)
           tma_load_3d(k_smem + ks * C::T_BYTES + hf * C::T_HALF, &tmK, &bars->k_full[ks],
                       hf * 64, j * BLK, b * p.Hkv + kvh);
         ++issued_k;
+        if (SKIPV) continue;   // warp 10 loads V
         const int vs = t % C::VST;
         if (!mbar_wait(&bars->v_empty[vs], ((t / C::VST) & 1) ^ 1, abort, lim)) break;
         mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
@@ -213,6 +223,30 @@ __global__ void __launch_bounds__(320, 1)
         for (int t = (issued_v > C::VST ? issued_v - C::VST : 0); t < issued_v; ++t)
           mbar_wait_drain(&bars->v_full[t % C::VST], (t / C::VST) & 1, lim);
       }
+    }
+  } else if (SKIPV && warp == 10) {
+    // ======================================================== V producer (V skipping)
+    if (lane == 0 && n > 0) {
+      prefetch_tensormap(&tmV);
+      int vc = 0;   // V tiles loaded
+      for (int t = 0; t < n; ++t) {
+        const int dq = t % C::DQ;
+        if (!mbar_wait(&bars->dq_full[dq], (t / C::DQ) & 1, abort, lim)) break;
+        const bool need = *reinterpret_cast<volatile int*>(&bars->dval[dq]) != 0;
+        mbar_arrive(&bars->dq_empty[dq]);
+        if (!need) continue;
+        const int vs = vc % C::VST;
+        if (!mbar_wait(&bars->v_empty[vs], ((vc / C::VST) & 1) ^ 1, abort, lim)) break;
+        mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
+        const int j = col_at(t);
+        for (int hf = 0; hf < C::HALVES; ++hf)
+          tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
+                      hf * 64, j * BLK, b * p.Hkv + kvh);
+        ++vc;
+      }
+      if (*abort)
+        for (int x = (vc > C::VST ? vc - C::VST : 0); x < vc; ++x)
+          mbar_wait_drain(&bars->v_full[x % C::VST], (x / C::VST) & 1, lim);
     }
   } else if (warp == 1) {
     // ======================================================== MMA issuer
@@ -248,8 +282,11 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         tl_mark(t, 1);
         const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[sb]);
-        const int vs = t % C::VST;
-        if (!mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) break;
+        // V ring position: every visited tile's, or (V skipping) the kept ones'
+        const int vi = SKIPV ? kept : t;
+        const int vs = vi % C::VST;
+        if ((!SKIPV || !skip) && !mbar_wait(&bars->v_full[vs], (vi / C::VST) & 1, abort, lim))
+          break;
         tc_fence_after();
         if (!skip) {
           const uint32_t p_tmem = tmem + C::S_COL + (uint32_t)sb * 128u;
@@ -263,7 +300,7 @@ __global__ void __launch_bounds__(320, 1)
           mma_commit(&bars->v_empty[vs]);
           tl_mark(t, 2);
           ++kept;
-        } else {
+        } else if (!SKIPV) {
           mbar_arrive(&bars->v_empty[vs]);
         }
         if (tr0) trace_mark(p.trace, p.trace_n, 2, t + 1);
@@ -375,6 +412,19 @@ __global__ void __launch_bounds__(320, 1)
       if (p.use_skip) {
         volatile int* vv = bars->vote[t & 1];
         skip = vv[0] & vv[1] & vv[2] & vv[3] & vv[4] & vv[5] & vv[6] & vv[7];
+      }
+      if (SKIPV) {   // the decision to the V producer, before any exponential
+        if (sw == 0 && lane == 0) {
+          const int dq = t % C::DQ;
+          if (mbar_wait(&bars->dq_empty[dq], ((t / C::DQ) & 1) ^ 1, abort, lim)) {
+            bars->dval[dq] = skip ? 0 : 1;
+            mbar_arrive(&bars->dq_full[dq]);
+          }
+        }
+        if (__any_sync(0xffffffffu, *abort != 0)) {
+          ok = false;
+          break;
+        }
       }
       const float mt = fmaxf(mth, xmax[((t & 1) * 2 + (half ^ 1)) * 128 + row]);
       m_run = fmaxf(m_run, mt);
@@ -502,16 +552,23 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
+template <int D, int BLK, bool SKIPV>
+static cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                              const PrefillParams& p, int grid, cudaStream_t stream) {
+  using C = PrefillCfg<D, BLK>;
+  static_assert(C::SMEM <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, BLK, SKIPV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  prefill_kernel<D, BLK, SKIPV><<<grid, SKIPV ? 352 : 320, C::SMEM, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
 template <int D, int BLK>
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const PrefillParams& p, int grid, cudaStream_t stream) {
-  using C = PrefillCfg<D, BLK>;
-  static_assert(C::SMEM <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, BLK>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return e;
-  prefill_kernel<D, BLK><<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  return p.skip_v ? launch_one<D, BLK, true>(tq, tk, tv, p, grid, stream)
+                  : launch_one<D, BLK, false>(tq, tk, tv, p, grid, stream);
 }
 
 template cudaError_t launch_prefill<128, 128>(const CUtensorMap&, const CUtensorMap&,

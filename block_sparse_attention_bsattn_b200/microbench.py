@@ -101,6 +101,9 @@ def main():
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--no-order", action="store_true", help="static masks: no longest-first order")
+    ap.add_argument("--reverse", action="store_true", help="prefill: descending visit order")
+    ap.add_argument("--skip-v", action="store_true", help="prefill: load V only for kept tiles")
+    ap.add_argument("--sink-seed", action="store_true", help="decode: sink-seeded splits")
     args = ap.parse_args()
     torch.cuda.set_device(0)
     out = {"what": args.what}
@@ -110,14 +113,17 @@ def main():
         lam = inputs.lambda_for(args.a, args.n)
         nq = args.n // 128
         st = torch.zeros(1, args.heads, nq, nq, dtype=torch.uint8, device="cuda")
-        o, _ = ops.bsattn_fwd_prefill(q, k, v, 128, None, True, lam, tile_status=st)
+        opt = dict(reverse=args.reverse, skip_v=args.skip_v)
+        o, _ = ops.bsattn_fwd_prefill(q, k, v, 128, None, True, lam, tile_status=st, **opt)
         torch.cuda.synchronize()
         vis, exe = int((st > 0).sum()), int((st == 2).sum())
-        fn = lambda: ops.bsattn_fwd_prefill(q, k, v, 128, None, True, lam, o=o, want_lse=False)
+        fn = lambda: ops.bsattn_fwd_prefill(q, k, v, 128, None, True, lam, o=o, want_lse=False,
+                                            **opt)
         for _ in range(args.warmup):
             fn()
         ms = _time(fn, args.iters)
-        out.update(heads=args.heads, n=args.n, a=args.a, visited=vis, executed=exe, ms=ms,
+        out.update(heads=args.heads, n=args.n, a=args.a, reverse=args.reverse,
+                   skip_v=args.skip_v, visited=vis, executed=exe, ms=ms,
                    tflops=TILE * (vis + exe) / ms / 1e9)
     elif args.what in ("videodit", "mmdit"):
         w = inputs.workload(args.what, device="cuda", generate=False)
@@ -145,16 +151,17 @@ def main():
         st = torch.zeros(B, Hkv, T, dtype=torch.uint8, device="cuda")
         ws = torch.empty(ops.bsattn_decode_workspace_size(B, Hq, d, ns), dtype=torch.uint8,
                          device="cuda")
-        o, _ = ops.bsattn_fwd_decode(q, k, v, 128, ns, None, lam, workspace=ws, tile_status=st)
+        o, _ = ops.bsattn_fwd_decode(q, k, v, 128, ns, None, lam, workspace=ws, tile_status=st,
+                                     sink_seed=args.sink_seed)
         torch.cuda.synchronize()
         vis, exe = int((st > 0).sum()), int((st == 2).sum())
         fn = lambda: ops.bsattn_fwd_decode(q, k, v, 128, ns, None, lam, o=o, want_lse=False,
-                                           workspace=ws)
+                                           workspace=ws, sink_seed=args.sink_seed)
         for _ in range(args.warmup):
             fn()
         ms = _time(fn, args.iters)
         byt = 2 * B * Hq * d * 2 + 128 * d * 2 * (vis + exe)
-        out.update(batch=B, l=L, hkv=Hkv, splits=ns, a=args.a, visited=vis, executed=exe, ms=ms, gbs=byt / ms / 1e6)
+        out.update(batch=B, l=L, hkv=Hkv, splits=ns, sink_seed=args.sink_seed, a=args.a, visited=vis, executed=exe, ms=ms, gbs=byt / ms / 1e6)
     print(json.dumps(out), flush=True)
 
 

@@ -59,6 +59,7 @@ _lib.bsattn_fwd_decode_noalloc.restype = _I
 
 # option bits of the _ex entry points (include/bsattn.h)
 PREFILL_REVERSE = 0x1
+PREFILL_SKIP_V = 0x2
 DECODE_SINK_SEED = 0x1
 
 EXPORTED = ("bsattn_status_string", "bsattn_version", "bsattn_debug_set", "bsattn_debug_trace",
@@ -152,10 +153,11 @@ def bsattn_fwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
                        want_lse: bool = True, tile_status: Optional[torch.Tensor] = None,
                        status: Optional[torch.Tensor] = None,
                        row_order: Optional[torch.Tensor] = None, stream=None,
-                       reverse: bool = False):
+                       reverse: bool = False, skip_v: bool = False):
     """q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 -> (o [B,Hq,N,d] bf16, lse [B,Hq,N] fp32 or None).
-    reverse: visit each row's key tiles in descending order (calls
-    bsattn_fwd_prefill_ex with BSATTN_PREFILL_REVERSE)."""
+    reverse: visit each row's key tiles in descending order; skip_v: load V
+    only for executed tiles (bsattn_fwd_prefill_ex with BSATTN_PREFILL_REVERSE
+    / BSATTN_PREFILL_SKIP_V)."""
     _check(q, "q", torch.bfloat16, 4)
     _check(k, "k", torch.bfloat16, 4)
     _check(v, "v", torch.bfloat16, 4)
@@ -172,7 +174,7 @@ def bsattn_fwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, int(block),
             float(scale), int(causal), float(lam), _ptr(row_ptr), _ptr(col_idx), _ptr(row_order),
             int(mask_heads), _ptr(tile_status))
-    flags = PREFILL_REVERSE if reverse else 0
+    flags = (PREFILL_REVERSE if reverse else 0) | (PREFILL_SKIP_V if skip_v else 0)
     if flags:
         rc = _lib.bsattn_fwd_prefill_ex(*args, flags, _ptr(status), _stream(stream))
     else:

@@ -147,6 +147,7 @@ int bsattn_fwd_prefill(const void *q, const void *k, const void *v, void *o, flo
 
 /* Option bits of bsattn_fwd_prefill_ex. */
 #define BSATTN_PREFILL_REVERSE 0x1u
+#define BSATTN_PREFILL_SKIP_V 0x2u
 
 /*
  * bsattn_fwd_prefill_ex -- bsattn_fwd_prefill with option bits; flags = 0 is
@@ -160,6 +161,13 @@ int bsattn_fwd_prefill(const void *q, const void *k, const void *v, void *o, flo
  * farther tiles are tested against it.  The skip decisions -- and so O, LSE
  * and tile_status -- are those of the reversed order; with lambda = 0 only
  * the summation order changes.
+ *
+ * BSATTN_PREFILL_SKIP_V: a V tile is loaded only when some query tile that
+ * shares it executes it, instead of for every visited tile.  Results are
+ * unchanged.  The BLASST page's prefill kernel loads every V tile (section
+ * 4.1: bandwidth is not the bottleneck, and a load issued after the decision
+ * cannot hide its latency) and names this as the option for memory-bound
+ * cases; it halves the bytes of a skipped step and delays every executed one.
  */
 int bsattn_fwd_prefill_ex(const void *q, const void *k, const void *v, void *o, float *lse,
                           int B, int Hq, int Hkv, int N, int d, int block, float scale,

@@ -112,7 +112,7 @@ def test_option_bits_validation(lib):
         return lib.bsattn_fwd_decode_ex(P(q) if q else None, P(0x2000), P(0x3000), P(0x4000),
                                         None, 2, 8, 2, 1000, 128, 128, 0.1, 0, 0.0, 4, P(0x9000),
                                         1 << 30, None, flags, None, None)
-    assert pre(0x2) == -1 and pre(0x80000000) == -1
+    assert pre(0x4) == -1 and pre(0x80000000) == -1
     assert pre(0x1, q=0) == -1
     assert dec(0x2) == -1 and dec(0x1, q=0) == -1
 

@@ -18,7 +18,7 @@ def _ops():
     return ops
 
 
-def _run_gpu(w, lam, mask=None, mask_heads=1, ordered=True, reverse=False):
+def _run_gpu(w, lam, mask=None, mask_heads=1, ordered=True, reverse=False, skip_v=False):
     """Index (with the longest-first row order unless `ordered` is False) and
     prefill through the C ABI; returns (o, lse, tile_status)."""
     ops = _ops()
@@ -34,14 +34,14 @@ def _run_gpu(w, lam, mask=None, mask_heads=1, ordered=True, reverse=False):
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     o, lse = ops.bsattn_fwd_prefill(q, k, v, w.block, w.scale, w.causal, lam, rp, ci, mask_heads,
                                     tile_status=st, status=status, row_order=order,
-                                    reverse=reverse)
+                                    reverse=reverse, skip_v=skip_v)
     torch.cuda.synchronize()
     assert status.item() == 0, ops.bsattn_status_string(status.item())
     return o, lse, st
 
 
-def _check(w, lam, mask=None, what="", ordered=True, reverse=False):
-    o, lse, st = _run_gpu(w, lam, mask, ordered=ordered, reverse=reverse)
+def _check(w, lam, mask=None, what="", ordered=True, reverse=False, skip_v=False):
+    o, lse, st = _run_gpu(w, lam, mask, ordered=ordered, reverse=reverse, skip_v=skip_v)
     ref = oracle.prefill(w.q, w.k, w.v, w.block, w.scale, w.causal, lam, mask=mask,
                          reverse=reverse)
     compare_outputs(o, ref["o"], lse, ref["lse"], what)
@@ -161,6 +161,52 @@ def test_reverse_visit_order_with_masks(block):
         m = (rng.random((heads, nb, nb)) < 0.6).astype(np.uint8)
         m[:, np.arange(nb), np.arange(nb)] = 1
         _check(w, 0.02, m, f"reverse mask{heads}", reverse=True)
+
+
+@pytest.mark.parametrize("hq,hkv,block,causal,masked", [
+    (4, 2, 128, True, False),    # two heads of one KV head per CTA
+    (1, 1, 128, True, False),    # two consecutive query tiles per CTA
+    (2, 1, 128, False, False),
+    (2, 1, 64, True, False),     # one query tile per CTA
+    (4, 2, 128, True, True),     # per-head masks: one query tile per CTA
+])
+@pytest.mark.parametrize("reverse", [False, True])
+def test_skip_v_loads(hq, hkv, block, causal, masked, reverse):
+    """V tiles loaded only for executed tiles: the results are those of the
+    oracle (which has no notion of loads) in either visit order."""
+    N = 6 * block + 45
+    q, k, v = inputs.blasst_prefill_qkv(1, hq, hkv, N, 128, "cpu", 77 + block)
+    w = inputs.Workload("skipv", 1, hq, hkv, N, 128, block, causal, "prefill",
+                        1 / math.sqrt(128), None, q=q, k=k, v=v)
+    mask = None
+    if masked:
+        nb = -(-N // block)
+        rng = np.random.default_rng(3)
+        mask = (rng.random((hq, nb, nb)) < 0.7).astype(np.uint8)
+        mask[:, np.arange(nb), np.arange(nb)] = 1
+    ref = _check(w, 0.02, mask, f"skip_v h{hq}/{hkv} b{block} rev{reverse}", reverse=reverse,
+                 skip_v=True)
+    if not reverse:
+        assert (ref["status"] == 1).sum() > 0
+
+
+def test_skip_v_dense_and_full_size_sampled():
+    """lambda = 0 with V skipping (every V tile is needed), and the full-size
+    BLASST prefill with V skipping on sampled query tiles."""
+    w = inputs.workload("blasst_prefill", shrink=True)
+    _check(w, 0.0, None, "skip_v dense", skip_v=True)
+    w = inputs.workload("blasst_prefill", device="cuda")
+    lam = inputs.lambda_for(10.0, w.N)
+    o, lse, st = _run_gpu(w, lam, None, skip_v=True)
+    items = _sampled_items(w, 12, 9)
+    ref = oracle.prefill(w.q.cpu(), w.k.cpu(), w.v.cpu(), w.block, w.scale, w.causal, lam,
+                         items=items)
+    o_c, lse_c, st_c = o.float().cpu().numpy(), lse.cpu().numpy(), st.cpu().numpy()
+    for (b, h, i) in items:
+        rows = slice(i * w.block, min(w.N, (i + 1) * w.block))
+        compare_outputs(o_c[b, h, rows], ref["o"][b, h, rows], lse_c[b, h, rows],
+                        ref["lse"][b, h, rows], f"skip_v item {(b, h, i)}")
+        compare_status(st_c[b, h, i], ref["status"][b, h, i], ref["margin"][b, h, i])
 
 
 def test_short_sequence_single_partial_tile():
