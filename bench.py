@@ -145,6 +145,7 @@ class Step:
         from block_sparse_attention_bsattn_b200 import inputs, ops
         self.ops = ops
         self.pw, self.dw, self.mask = pw, dw, mask
+        self.opts = {"reverse": False, "skip_v": False, "sink_seed": False}
         self.set_a(a)
         nb = pw.nq
         self.row_ptr = torch.empty(nb + 1, dtype=torch.int32, device="cuda")
@@ -180,13 +181,15 @@ class Step:
         self.ops.bsattn_fwd_prefill(pw.q, pw.k, pw.v, BLK, pw.scale, True, self.p_lam,
                                     self.row_ptr, self.col_idx, 1, o=self.o, lse=self.lse,
                                     tile_status=tile_status, status=self.status,
-                                    row_order=self.row_order)
+                                    row_order=self.row_order, reverse=self.opts["reverse"],
+                                    skip_v=self.opts["skip_v"])
 
     def decode(self, tile_status=None):
         dw = self.dw
         self.ops.bsattn_fwd_decode(dw.q, dw.k, dw.v, BLK, dw.num_splits, dw.scale, self.d_lam,
                                    o=self.do, lse=self.dlse, workspace=self.ws,
-                                   tile_status=tile_status, status=self.status)
+                                   tile_status=tile_status, status=self.status,
+                                   sink_seed=self.opts["sink_seed"])
 
     LAUNCHES = 4 + 1 + 2
 
@@ -428,6 +431,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-variants", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -499,6 +503,32 @@ def main():
             })
         step.set_a(args.a)
 
+    # the options of the _ex entry points at the same a: descending visit
+    # order and V skipping (prefill), sink-seeded splits (decode)
+    variants = {}
+    if not args.no_variants:
+        for name, opt, phase in (("prefill_reverse", "reverse", "prefill"),
+                                 ("prefill_skip_v", "skip_v", "prefill"),
+                                 ("decode_sink_seed", "sink_seed", "decode")):
+            step.opts[opt] = True
+            c = step.counts()
+            for _ in range(2):
+                step.index(); getattr(step, phase)()
+            n = max(3, K // 4)
+            sp, _ = timed_phases(step, n, ("index", phase))
+            ms = max_over_ranks(sp[phase]) / n
+            if phase == "prefill":
+                variants[name] = {"ms": ms, "tflops": prefill_flops(c) / (ms * 1e-3) / 1e12,
+                                  "skipped_frac": 1 - c["p_executed"] / c["p_visited"],
+                                  "vs_default_ms": p_ms}
+            else:
+                variants[name] = {"ms": ms, "gbs": decode_bytes(dw, c) / (ms * 1e-3) / 1e9,
+                                  "skipped_frac": 1 - c["d_executed"] / c["d_visited"],
+                                  "vs_default_ms": d_ms,
+                                  "note": "bytes exclude the one extra K tile per split read "
+                                          "to seed the running max"}
+            step.opts[opt] = False
+
     e2e = None
     if not args.no_e2e:
         e_p_ms, e_d_ms, byts = e2e_run(step, max(3, K // 2))
@@ -566,6 +596,7 @@ def main():
         "sparsity": {"prefill_skipped_frac": 1 - counts["p_executed"] / counts["p_visited"],
                      "decode_skipped_frac": 1 - counts["d_executed"] / counts["d_visited"]},
         "sweep": sweep,
+        "variants": variants,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": Step.LAUNCHES * K,
