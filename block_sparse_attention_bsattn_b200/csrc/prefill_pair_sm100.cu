@@ -411,15 +411,7 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
           if (key >= p.N || (p.causal && key > qpos)) r[c] = __float_as_uint(-INFINITY);
         }
       }
-      float m8[8];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) m8[x] = __uint_as_float(r[x]);
-#pragma unroll
-      for (int c = 8; c < BLK; c += 8)
-#pragma unroll
-        for (int x = 0; x < 8; ++x) m8[x] = fmaxf(m8[x], __uint_as_float(r[c + x]));
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      const float mx = row_max<BLK>(reinterpret_cast<const float*>(r));
       const float mt = mx * p.scale_log2;
       int skip = 0;
       if (p.use_skip) {

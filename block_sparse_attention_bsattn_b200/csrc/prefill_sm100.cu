@@ -383,15 +383,7 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
             if (key >= p.N || (p.causal && key > qpos)) s[c] = -INFINITY;
           }
         }
-        float m8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) m8[e] = s[e];
-#pragma unroll
-        for (int c = 8; c < CW; c += 8)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], s[c + e]);
-        mh = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        mh = row_max<CW>(s);
       }
       const float mth = mh * p.scale_log2;  // half-row max, base-2 units
       // The row passes iff both of its halves pass: max(a, b) - m < t exactly

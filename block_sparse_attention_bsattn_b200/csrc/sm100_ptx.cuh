@@ -244,6 +244,29 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// max of three floats in one instruction (sm_100's three-input max.f32)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Row max of N (a multiple of 16) fp32 values: eight independent
+// three-input chains, then a three-input tree.
+template <int N>
+__device__ __forceinline__ float row_max(const float* v) {
+  static_assert(N % 16 == 0, "row_max");
+  float m[8];
+#pragma unroll
+  for (int x = 0; x < 8; ++x) m[x] = fmax3(v[x], v[8 + x], N > 16 ? v[16 + x] : -INFINITY);
+#pragma unroll
+  for (int c = 24; c < N; c += 16)
+#pragma unroll
+    for (int x = 0; x < 8; ++x) m[x] = fmax3(m[x], v[c + x], c + 8 < N ? v[c + 8 + x] : -INFINITY);
+  const float a = fmax3(m[0], m[1], m[2]), b = fmax3(m[3], m[4], m[5]);
+  return fmax3(a, b, fmaxf(m[6], m[7]));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
