@@ -56,10 +56,10 @@ def bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_build_index.argtypes = [P, i32, i32, i32, i32, i32, i32, P, P, i64, P]
     lib.oracle_build_index.restype = i32
     lib.oracle_prefill.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, i32,
-                                   f64, P, i32, P, i32, P, P, P, P, i32]
+                                   f64, P, i32, P, i32, P, P, P, P, i32, P]
     lib.oracle_prefill.restype = i32
     lib.oracle_decode.argtypes = [P, P, P, i32, i32, i64, i32, i32, f64, f64, i32,
-                                  P, P, P, P, i32]
+                                  P, P, P, P, i32, P]
     lib.oracle_decode.restype = i32
     lib.oracle_num_threads.restype = i32
     return lib
@@ -119,11 +119,13 @@ def build_index(mask: np.ndarray, q_block: int, k_block: int, causal: bool,
 
 
 def prefill(q, k, v, block: int, scale: float, causal: bool, lam: float,
-            mask=None, items=None, reverse: bool = False):
+            mask=None, items=None, reverse: bool = False, seq_lens=None):
     """Block-sparse prefill.  q [B,Hq,N,d], k/v [B,Hkv,N,d] (bf16 torch or
     uint16 bits).  mask: None or uint8 [Hm, nq, nk].  items: None or an int
     array of (b, h, i) rows.  reverse: visit each row's key tiles in
-    descending order (the BLASST page's block-row reordering).  Returns dict(o, lse, status, margin) with o
+    descending order (the BLASST page's block-row reordering).  seq_lens:
+    None or [B] valid lengths (key padding: keys and query rows at or past a
+    sequence's length are padding).  Returns dict(o, lse, status, margin) with o
     [B,Hq,N,d] f64, lse [B,Hq,N] f64, status uint8 [B,Hq,nq,nk] (0 = not
     visited, 1 = skipped, 2 = executed), margin f64 [B,Hq,nq,nk]."""
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
@@ -139,6 +141,9 @@ def prefill(q, k, v, block: int, scale: float, causal: bool, lam: float,
     if mask is not None:
         m = np.ascontiguousarray(mask, dtype=np.uint8)
         mh = m.shape[0]
+    sl = None
+    if seq_lens is not None:
+        sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32).reshape(B))
     it = None
     n_items = 0
     if items is not None:
@@ -147,17 +152,18 @@ def prefill(q, k, v, block: int, scale: float, causal: bool, lam: float,
     rc = _load().oracle_prefill(_ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, N, d, block,
                                 float(scale), int(causal), float(lam), _ptr(m), mh,
                                 _ptr(it), n_items, _ptr(o), _ptr(lse), _ptr(status),
-                                _ptr(margin), int(reverse))
+                                _ptr(margin), int(reverse), _ptr(sl))
     if rc != 0:
         raise OracleError(f"oracle_prefill rc={rc}")
     return {"o": o, "lse": lse, "status": status, "margin": margin}
 
 
 def decode(q, k, v, block: int, scale: float, lam: float, num_splits: int,
-           sink_seed: bool = False):
+           sink_seed: bool = False, lens=None):
     """Split-KV decode over independent problems.  q [n, g, d], k/v [n, L, d]
     (bf16 torch or uint16 bits).  sink_seed: every split after the first
-    starts its running max from key tile 0's row max.  Returns dict(o [n,g,d], lse [n,g],
+    starts its running max from key tile 0's row max.  lens: None or [n]
+    cache lengths (the splits cut each problem's own tiles).  Returns dict(o [n,g,d], lse [n,g],
     status uint8 [n,T], margin [n,T])."""
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     n, g, d = qb.shape
@@ -167,9 +173,12 @@ def decode(q, k, v, block: int, scale: float, lam: float, num_splits: int,
     lse = np.zeros((n, g), np.float64)
     status = np.zeros((n, T), np.uint8)
     margin = np.zeros((n, T), np.float64)
+    ln = None
+    if lens is not None:
+        ln = np.ascontiguousarray(np.asarray(lens, dtype=np.int64).reshape(n))
     rc = _load().oracle_decode(_ptr(qb), _ptr(kb), _ptr(vb), n, g, L, d, block, float(scale),
                                float(lam), num_splits, _ptr(o), _ptr(lse), _ptr(status),
-                               _ptr(margin), int(sink_seed))
+                               _ptr(margin), int(sink_seed), _ptr(ln))
     if rc != 0:
         raise OracleError(f"oracle_decode rc={rc}")
     return {"o": o, "lse": lse, "status": status, "margin": margin}

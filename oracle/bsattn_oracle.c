@@ -40,6 +40,13 @@
  *    request (sink seeding) every chunk but the first starts instead from the
  *    row max of key tile 0, the tile that holds the attention sink; tile 0 is
  *    then scored by that chunk but neither visited nor executed by it.
+ *  - Variable lengths (key padding, "块稀疏Attention实战" section 5.2: pad
+ *    the batch to its longest sequence and mask the padding keys): sequence b
+ *    has len_b valid tokens; keys at or past len_b take no part, key tiles
+ *    wholly past it are not visited, and query rows at or past it are padding
+ *    (no vote, O = 0, LSE = -inf).  A padded batch therefore equals every
+ *    sequence computed alone at its own length; in decode the splits cut the
+ *    sequence's own ceil(len_b / block) tiles.
  *  - The result is the exact softmax over the keys of the executed tiles,
  *    computed in two passes (max, then sum) -- algebraically what the online
  *    recurrence of Algorithm 1 reaches.
@@ -280,6 +287,7 @@ static void query_tile(const uint16_t *const *qrows, const int64_t *qpos, int nr
  * o: [B][Hq][N][d], lse: [B][Hq][N] (doubles); tile_status / margin:
  * NULL or [B][Hq][nq][nk].  Only rows of the listed items are written.
  * reverse: 0 visits each row's key tiles in ascending order, 1 in descending.
+ * seq_lens: NULL (every sequence has N tokens) or [B] valid lengths in [0, N].
  */
 int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                    int B, int Hq, int Hkv, int N, int d, int block,
@@ -287,7 +295,7 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                    const uint8_t *mask, int mask_heads,
                    const int32_t *items, int n_items,
                    double *o, double *lse, uint8_t *tile_status, double *margin,
-                   int reverse)
+                   int reverse, const int32_t *seq_lens)
 {
     if (!q || !k || !v || !o || !lse || B < 1 || Hq < 1 || Hkv < 1 ||
         Hq % Hkv != 0 || N < 1 || d < 1 || block < 1 ||
@@ -295,6 +303,10 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         return ORACLE_ERR_ARG;
     if (mask && mask_heads != 1 && mask_heads != Hq)
         return ORACLE_ERR_ARG;
+    if (seq_lens)
+        for (int b = 0; b < B; ++b)
+            if (seq_lens[b] < 0 || seq_lens[b] > N)
+                return ORACLE_ERR_ARG;
     const int g = Hq / Hkv;
     const int nq = (N + block - 1) / block, nk = nq;
     const int64_t total = items ? n_items : (int64_t)B * Hq * nq;
@@ -313,7 +325,16 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         }
         const int kvh = h / g;
         const int64_t r0 = (int64_t)i * block;
-        const int nrows = (int)((r0 + block <= N) ? block : N - r0);
+        const int nrows_all = (int)((r0 + block <= N) ? block : N - r0);
+        const int64_t len = seq_lens ? seq_lens[b] : N;
+        /* rows at or past the sequence's length are padding */
+        const int nrows = r0 >= len ? 0 : (int)((r0 + nrows_all <= len) ? nrows_all : len - r0);
+        for (int r = nrows; r < nrows_all; ++r) {
+            double *orow_pad = o + (((int64_t)b * Hq + h) * N + r0 + r) * d;
+            for (int x = 0; x < d; ++x)
+                orow_pad[x] = 0.0;
+            lse[((int64_t)b * Hq + h) * N + r0 + r] = -INFINITY;
+        }
         const uint16_t *qrows[1024];
         int64_t qpos[1024];
         for (int r = 0; r < nrows; ++r) {
@@ -327,6 +348,8 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             if (mask && !mask[((int64_t)mh * nq + i) * nk + j])
                 continue;
             if (causal && (int64_t)j * block > (int64_t)(i + 1) * block - 1)
+                continue;
+            if ((int64_t)j * block >= len)   /* wholly padding keys */
                 continue;
             tiles[nt++] = j;
         }
@@ -342,7 +365,9 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         const uint16_t *vb = v + ((int64_t)b * Hkv + kvh) * N * d;
         double *orow = o + (((int64_t)b * Hq + h) * N + r0) * d;
         double *lrow = lse + ((int64_t)b * Hq + h) * N + r0;
-        query_tile(qrows, qpos, nrows, kb, vb, N, d, block, scale, causal, lambda,
+        if (nrows == 0)
+            nt = 0;   /* a query tile of padding only visits nothing */
+        query_tile(qrows, qpos, nrows, kb, vb, len, d, block, scale, causal, lambda,
                    tiles, NULL, nt, -1, orow, lrow, st, mg);
         int64_t sbase = (((int64_t)b * Hq + h) * nq + i) * nk;
         for (int t = 0; t < nt; ++t) {
@@ -364,38 +389,48 @@ int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v,
  * o: [n][g][d], lse: [n][g]; tile_status / margin: NULL or [n][T] with
  * T = ceil(L / block).  A single query at the last position sees all L keys.
  * sink_seed: 1 starts every split after the first from key tile 0's row max.
+ * lens: NULL (every cache holds L tokens) or [n_problems] lengths in [0, L];
+ *       problem p's splits cut its own ceil(lens[p] / block) tiles.
  */
 int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                   int n_problems, int g, int64_t L, int d, int block,
                   double scale, double lambda, int num_splits,
                   double *o, double *lse, uint8_t *tile_status, double *margin,
-                  int sink_seed)
+                  int sink_seed, const int64_t *lens)
 {
     if (!q || !k || !v || !o || !lse || n_problems < 1 || g < 1 || g > 1024 ||
         L < 1 || d < 1 || block < 1 || num_splits < 1 ||
         !(lambda >= 0.0 && lambda <= 1.0))
         return ORACLE_ERR_ARG;
     const int T = (int)((L + block - 1) / block);
-    const int chunk = (T + num_splits - 1) / num_splits;
+    if (lens)
+        for (int p = 0; p < n_problems; ++p)
+            if (lens[p] < 0 || lens[p] > L)
+                return ORACLE_ERR_ARG;
 
 #pragma omp parallel for schedule(dynamic, 1)
     for (int p = 0; p < n_problems; ++p) {
+        const int64_t Lp = lens ? lens[p] : L;
+        const int Tp = (int)((Lp + block - 1) / block);
+        const int chunk = Tp > 0 ? (Tp + num_splits - 1) / num_splits : 1;
         const uint16_t *qrows[1024];
         int64_t qpos[1024];
         for (int r = 0; r < g; ++r) {
             qrows[r] = q + ((int64_t)p * g + r) * d;
-            qpos[r] = L - 1;
+            qpos[r] = Lp - 1;
         }
-        int32_t *tiles = malloc(sizeof(int32_t) * T);
-        uint8_t *starts = malloc(T);
-        for (int t = 0; t < T; ++t) {
+        int32_t *tiles = malloc(sizeof(int32_t) * (T > 0 ? T : 1));
+        uint8_t *starts = malloc(T > 0 ? T : 1);
+        for (int t = 0; t < Tp; ++t) {
             tiles[t] = t;
             starts[t] = (t % chunk) == 0;
         }
-        uint8_t *st = malloc(T);
-        double *mg = malloc(sizeof(double) * T);
-        query_tile(qrows, qpos, g, k + (int64_t)p * L * d, v + (int64_t)p * L * d, L,
-                   d, block, scale, 0, lambda, tiles, starts, T, sink_seed ? 0 : -1,
+        uint8_t *st = calloc(T > 0 ? T : 1, 1);
+        double *mg = malloc(sizeof(double) * (T > 0 ? T : 1));
+        for (int t = 0; t < T; ++t)
+            mg[t] = NAN;
+        query_tile(qrows, qpos, g, k + (int64_t)p * L * d, v + (int64_t)p * L * d, Lp,
+                   d, block, scale, 0, lambda, tiles, starts, Tp, sink_seed ? 0 : -1,
                    o + (int64_t)p * g * d, lse + (int64_t)p * g, st, mg);
         for (int t = 0; t < T; ++t) {
             if (tile_status)

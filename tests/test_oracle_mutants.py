@@ -32,6 +32,10 @@ MUTANTS = {
     "reverse_ignored": [("        if (reverse)\n", "        if (0)\n")],
     "seed_ignored": [("if (seed_tile >= 0 && tiles[t] != seed_tile)", "if (0)")],
     "seed_from_split_first_tile": [("SCORE_TILE(seed_tile);", "SCORE_TILE(tiles[t]);")],
+    "padding_keys_not_masked": [("query_tile(qrows, qpos, nrows, kb, vb, len, d,",
+                                 "query_tile(qrows, qpos, nrows, kb, vb, N, d,")],
+    "decode_splits_cut_full_cache": [("const int chunk = Tp > 0 ? (Tp + num_splits - 1) / num_splits : 1;",
+                                      "const int chunk = (T + num_splits - 1) / num_splits;")],
 }
 
 CHECKS = [
@@ -44,6 +48,8 @@ CHECKS = [
     pins.test_closed_form_order_matters,
     pins.test_closed_form_reverse_order,
     pins.test_decode_sink_seed_closed_form,
+    lambda: pins.test_varlen_prefill_equals_each_sequence_alone(False, True, 1e-2),
+    pins.test_varlen_decode_equals_each_cache_alone,
     pins.test_decode_split_resets_running_max,
     pins.test_decode_gqa_group_vote,
     pins.test_index_matches_definition_and_causal,

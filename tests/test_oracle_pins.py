@@ -376,6 +376,70 @@ def test_decode_sink_seed_only_adds_skips():
     assert np.abs(a0["o"] - b0["o"]).max() == 0.0
 
 
+@pytest.mark.parametrize("causal,masked,lam", [(True, False, 0.0), (True, False, 2e-2),
+                                               (False, True, 1e-2), (True, True, 5e-2)])
+def test_varlen_prefill_equals_each_sequence_alone(causal, masked, lam):
+    """Key padding (the multimodal DiT page, section 5.2): a batch padded to
+    N with valid lengths len_b gives, for every sequence, exactly what the
+    sequence gives alone at N = len_b (same O, LSE, executed tiles), and its
+    padding rows get O = 0 and LSE = -inf."""
+    B, Hq, Hkv, N, d, block = 4, 4, 2, 5 * 64 + 9, 64, 64
+    lens = [N, 200, 64, 0]
+    q, k, v = inputs.blasst_prefill_qkv(B, Hq, Hkv, N, d, "cpu", 17)
+    nb = -(-N // block)
+    mask = None
+    if masked:
+        rng = np.random.default_rng(4)
+        mask = (rng.random((1, nb, nb)) < 0.6).astype(np.uint8)
+        mask[0, np.arange(nb), np.arange(nb)] = 1
+    r = oracle.prefill(q, k, v, block, 0.125, causal, lam, mask=mask, seq_lens=lens)
+    for b, L in enumerate(lens):
+        if L > 0:
+            nl = -(-L // block)
+            m = None if mask is None else np.ascontiguousarray(mask[:, :nl, :nl])
+            alone = oracle.prefill(q[b:b + 1, :, :L], k[b:b + 1, :, :L], v[b:b + 1, :, :L], block,
+                                   0.125, causal, lam, mask=m)
+            assert np.abs(r["o"][b, :, :L] - alone["o"][0]).max() < 1e-12
+            assert np.abs(r["lse"][b, :, :L] - alone["lse"][0]).max() < 1e-12
+            assert (r["status"][b, :, :nl, :nl] == alone["status"][0]).all()
+            assert (r["status"][b, :, :, nl:] == 0).all() and (r["status"][b, :, nl:] == 0).all()
+        assert (r["o"][b, :, L:] == 0).all()
+        assert np.isneginf(r["lse"][b, :, L:]).all()
+
+
+def test_varlen_decode_equals_each_cache_alone():
+    """Decode with per-sequence cache lengths: each problem equals its cache
+    truncated to its own length, split by the same num_splits."""
+    n, g, L, d, block = 5, 4, 23 * 64 + 7, 64, 64
+    lens = [L, 1000, 64, 1, 0]
+    q, k, v = inputs.blasst_decode_qkv(1, n * g, n, L, d, "cpu", 18)
+    qs, ks, vs = oracle.decode_problems(q, k, v, [(0, x) for x in range(n)])
+    for seed in (False, True):
+        r = oracle.decode(qs, ks, vs, block, 0.125, 1e-2, 4, sink_seed=seed, lens=lens)
+        for p, Lp in enumerate(lens):
+            if Lp == 0:
+                assert (r["o"][p] == 0).all() and np.isneginf(r["lse"][p]).all()
+                assert (r["status"][p] == 0).all()
+                continue
+            alone = oracle.decode(qs[p:p + 1], ks[p:p + 1, :Lp], vs[p:p + 1, :Lp], block, 0.125,
+                                  1e-2, 4, sink_seed=seed)
+            Tp = -(-Lp // block)
+            assert np.abs(r["o"][p] - alone["o"][0]).max() < 1e-12
+            assert np.abs(r["lse"][p] - alone["lse"][0]).max() < 1e-12
+            assert (r["status"][p, :Tp] == alone["status"][0]).all()
+            assert (r["status"][p, Tp:] == 0).all()
+    # closed form: a cache of 4 tiles inside a buffer of 8, two splits.  Its own
+    # tiles split {0, 1} {2, 3}: tile 2 starts a split and is executed, and
+    # tile 3 ties it; the buffer's tiles would have split {0..3} and skipped
+    # tiles 1..3 (score 0, 10 below key 0's)
+    d1, blk = 64, 64
+    q1 = np.zeros((1, 1, d1)); q1[0, 0, 0] = 1.0
+    k1 = np.zeros((1, 8 * blk, d1)); k1[0, 0, 0] = 10.0
+    v1 = np.random.default_rng(5).integers(-4, 5, (1, 8 * blk, d1)).astype(np.float64)
+    r1 = oracle.decode(_bf16(q1), _bf16(k1), _bf16(v1), blk, 1.0, math.exp(-5), 2, lens=[4 * blk])
+    assert list(r1["status"][0]) == [2, 1, 2, 2, 0, 0, 0, 0]
+
+
 def test_decode_gqa_group_vote():
     """Decode query tile = the g query heads of one KV head; a V tile is skipped
     only when all g heads pass."""
