@@ -145,7 +145,7 @@ class Step:
         from block_sparse_attention_bsattn_b200 import inputs, ops
         self.ops = ops
         self.pw, self.dw, self.mask = pw, dw, mask
-        self.opts = {"reverse": False, "skip_v": False, "sink_seed": False}
+        self.opts = {"reverse": False, "skip_v": False, "sink_seed": False, "seq_lens": None}
         self.set_a(a)
         nb = pw.nq
         self.row_ptr = torch.empty(nb + 1, dtype=torch.int32, device="cuda")
@@ -189,7 +189,7 @@ class Step:
         self.ops.bsattn_fwd_decode(dw.q, dw.k, dw.v, BLK, dw.num_splits, dw.scale, self.d_lam,
                                    o=self.do, lse=self.dlse, workspace=self.ws,
                                    tile_status=tile_status, status=self.status,
-                                   sink_seed=self.opts["sink_seed"])
+                                   sink_seed=self.opts["sink_seed"], seq_lens=self.opts["seq_lens"])
 
     LAUNCHES = 4 + 1 + 2
 
@@ -507,10 +507,14 @@ def main():
     # order and V skipping (prefill), sink-seeded splits (decode)
     variants = {}
     if not args.no_variants:
+        # cache lengths drawn uniformly from [L/8, L] (seeded): key padding
+        g = torch.Generator().manual_seed(4321 + rank)
+        varlen = torch.randint(dw.N // 8, dw.N + 1, (dw.B,), generator=g, dtype=torch.int32).cuda()
         for name, opt, phase in (("prefill_reverse", "reverse", "prefill"),
                                  ("prefill_skip_v", "skip_v", "prefill"),
-                                 ("decode_sink_seed", "sink_seed", "decode")):
-            step.opts[opt] = True
+                                 ("decode_sink_seed", "sink_seed", "decode"),
+                                 ("decode_varlen", "seq_lens", "decode")):
+            step.opts[opt] = varlen if opt == "seq_lens" else True
             c = step.counts()
             for _ in range(2):
                 step.index(); getattr(step, phase)()
@@ -526,8 +530,10 @@ def main():
                                   "skipped_frac": 1 - c["d_executed"] / c["d_visited"],
                                   "vs_default_ms": d_ms,
                                   "note": "bytes exclude the one extra K tile per split read "
-                                          "to seed the running max"}
-            step.opts[opt] = False
+                                          "to seed the running max" if opt == "sink_seed" else
+                                          "cache lengths uniform in [L/8, L]; bytes count the "
+                                          "valid tiles only"}
+            step.opts[opt] = None if opt == "seq_lens" else False
 
     e2e = None
     if not args.no_e2e:

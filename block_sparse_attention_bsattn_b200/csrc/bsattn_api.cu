@@ -158,16 +158,16 @@ int bsattn_fwd_prefill(const void* q, const void* k, const void* v, void* o, flo
                        const int32_t* row_order, int mask_heads, uint8_t* tile_status,
                        int32_t* d_status, cudaStream_t stream) {
   return bsattn_fwd_prefill_ex(q, k, v, o, lse, B, Hq, Hkv, N, d, block, scale, causal, lambda,
-                               row_ptr, col_idx, row_order, mask_heads, tile_status, 0u,
-                               d_status, stream);
+                               row_ptr, col_idx, row_order, mask_heads, tile_status, nullptr,
+                               0u, d_status, stream);
 }
 
 int bsattn_fwd_prefill_ex(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int Hq, int Hkv, int N, int d, int block, float scale,
                           int causal, float lambda, const int32_t* row_ptr,
                           const int32_t* col_idx, const int32_t* row_order, int mask_heads,
-                          uint8_t* tile_status, unsigned flags, int32_t* d_status,
-                          cudaStream_t stream) {
+                          uint8_t* tile_status, const int32_t* d_seq_lens, unsigned flags,
+                          int32_t* d_status, cudaStream_t stream) {
   if (!q || !k || !v || !o) return BSATTN_ERR_INVALID_ARG;
   if (flags & ~(BSATTN_PREFILL_REVERSE | BSATTN_PREFILL_SKIP_V)) return BSATTN_ERR_INVALID_ARG;
   if (row_order && !row_ptr) return BSATTN_ERR_INVALID_ARG;
@@ -215,6 +215,7 @@ int bsattn_fwd_prefill_ex(const void* q, const void* k, const void* v, void* o, 
   p.thr_log2 = lambda > 0.f ? (float)std::log2((double)lambda) : -INFINITY;
   p.reverse = (flags & BSATTN_PREFILL_REVERSE) ? 1 : 0;
   p.skip_v = (flags & BSATTN_PREFILL_SKIP_V) ? 1 : 0;
+  p.seq_lens = d_seq_lens;
   p.debug_stall = g_inject_stall;
   p.wait_limit_ns = g_wait_limit_ns;
   p.trace = g_trace;
@@ -251,15 +252,15 @@ int bsattn_fwd_decode(const void* q, const void* k, const void* v, void* o, floa
                       float lambda, int num_splits, void* workspace, size_t workspace_bytes,
                       uint8_t* tile_status, int32_t* d_status, cudaStream_t stream) {
   return bsattn_fwd_decode_ex(q, k, v, o, lse, B, Hq, Hkv, L, d, block, scale, causal, lambda,
-                              num_splits, workspace, workspace_bytes, tile_status, 0u, d_status,
-                              stream);
+                              num_splits, workspace, workspace_bytes, tile_status, nullptr, 0u,
+                              d_status, stream);
 }
 
 int bsattn_fwd_decode_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                          int Hq, int Hkv, int L, int d, int block, float scale, int causal,
                          float lambda, int num_splits, void* workspace, size_t workspace_bytes,
-                         uint8_t* tile_status, unsigned flags, int32_t* d_status,
-                         cudaStream_t stream) {
+                         uint8_t* tile_status, const int32_t* d_seq_lens, unsigned flags,
+                         int32_t* d_status, cudaStream_t stream) {
   (void)causal;
   if (!q || !k || !v || !o || !workspace) return BSATTN_ERR_INVALID_ARG;
   if (flags & ~BSATTN_DECODE_SINK_SEED) return BSATTN_ERR_INVALID_ARG;
@@ -309,6 +310,7 @@ int bsattn_fwd_decode_ex(const void* q, const void* k, const void* v, void* o, f
   p.use_skip = lambda > 0.f ? 1 : 0;
   p.thr_log2 = lambda > 0.f ? (float)std::log2((double)lambda) : -INFINITY;
   p.sink_seed = (flags & BSATTN_DECODE_SINK_SEED) ? 1 : 0;
+  p.seq_lens = d_seq_lens;
   p.wait_limit_ns = g_wait_limit_ns;
   p.trace = g_trace;
   p.trace_n = g_trace_n;

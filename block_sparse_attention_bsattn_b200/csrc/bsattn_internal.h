@@ -36,6 +36,7 @@ struct PrefillParams {
   int pair_tiles;    // two-slot kernel: consecutive query tiles of one head
   int reverse;       // visit each row's key tiles in descending order
   int skip_v;        // load V only for tiles some query tile keeps
+  const int32_t* seq_lens;   // [B] valid tokens per sequence (key padding) or null
   unsigned long long wait_limit_ns;
   volatile int32_t* trace;  // debug: progress markers (host-visible memory) or null
   int trace_n;
@@ -53,6 +54,7 @@ struct DecodeParams {
   float thr_log2;
   int use_skip;
   int sink_seed;    // splits after the first start from key tile 0's row max
+  const int32_t* seq_lens;   // [B] cache lengths (splits cut each one's own tiles) or null
   unsigned long long wait_limit_ns;
   volatile int32_t* trace;
   int trace_n;

@@ -113,8 +113,12 @@ __global__ void __launch_bounds__(256, 1)
   const int split = blockIdx.x % p.splits;
   const int bk = blockIdx.x / p.splits;
   const int b = bk / p.Hkv, kvh = bk % p.Hkv;
-  const int t_begin = split * p.chunk;
-  const int t_end = min(p.T, t_begin + p.chunk);
+  // cache length (the splits cut the sequence's own tiles) and tile range
+  const int lenb = p.seq_lens ? min(max(p.seq_lens[b], 0), p.L) : p.L;
+  const int Tb = p.seq_lens ? (lenb + BLK - 1) / BLK : p.T;
+  const int chunk = p.seq_lens ? (Tb > 0 ? (Tb + p.splits - 1) / p.splits : 1) : p.chunk;
+  const int t_begin = split * chunk;
+  const int t_end = min(Tb, t_begin + chunk);
   // tile stream of the split: with sink seeding, step 0 scores key tile 0
   // only to start the running max; step t >= sd is key tile t_begin + t - sd
   const int sd = (p.sink_seed && split > 0 && t_end > t_begin) ? 1 : 0;
@@ -208,7 +212,7 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
           for (int g = 0; g < G; ++g) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], off);
         const int kpos = tile_of(t) * BLK + key;
-        if (kpos >= p.L)
+        if (kpos >= lenb)
 #pragma unroll
           for (int g = 0; g < G; ++g) acc[g] = -INFINITY;
         // warp max over its KPW keys

@@ -151,15 +151,22 @@ __global__ void __launch_bounds__(224, 1)
 
   // item n of this CTA -> (batch, kv head, split) and its tile stream: nt
   // steps; with sink seeding (sd = 1) step 0 scores key tile 0 only to start
-  // the running max, and step t >= sd is key tile t0 + t - sd
+  // the running max, and step t >= sd is key tile t0 + t - sd.  With cache
+  // lengths the splits cut the sequence's own ceil(len / 128) tiles.
+  auto len_of = [&](int b) { return p.seq_lens ? min(max(p.seq_lens[b], 0), p.L) : p.L; };
   auto item_of = [&](int n, int& b, int& kvh, int& split, int& t0, int& nt, int& sd) {
     const int it = blockIdx.x + n * gridDim.x;
     split = it % p.splits;
     const int bk = it / p.splits;
     b = bk / p.Hkv;
     kvh = bk % p.Hkv;
-    t0 = split * p.chunk;
-    nt = max(0, min(p.T, t0 + p.chunk) - t0);
+    int T = p.T, chunk = p.chunk;
+    if (p.seq_lens) {
+      T = (len_of(b) + C::BLK - 1) / C::BLK;
+      chunk = T > 0 ? (T + p.splits - 1) / p.splits : 1;
+    }
+    t0 = split * chunk;
+    nt = max(0, min(T, t0 + chunk) - t0);
     sd = (p.sink_seed && split > 0 && nt > 0) ? 1 : 0;
     nt += sd;
   };
@@ -316,6 +323,7 @@ __global__ void __launch_bounds__(224, 1)
     for (int n = 0; ok && n < my_items; ++n) {
       int b, kvh, split, t0, nt, sd;
       item_of(n, b, kvh, split, t0, nt, sd);
+      const int lenb = len_of(b);
       float m_run[NC], m_ref[NC], lp[NC];
 #pragma unroll
       for (int c = 0; c < NC; ++c) { m_run[c] = -INFINITY; m_ref[c] = -INFINITY; lp[c] = 0.f; }
@@ -341,7 +349,7 @@ __global__ void __launch_bounds__(224, 1)
         if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
         const int jt = tile_of(t0, sd, t);
         const bool seed = sd && t == 0;
-        const bool key_ok = jt * C::BLK + key < p.L;
+        const bool key_ok = jt * C::BLK + key < lenb;
         float s[NC];
 #pragma unroll
         for (int c = 0; c < NC; ++c) s[c] = (key_ok && c < G) ? __uint_as_float(r[c]) : -INFINITY;

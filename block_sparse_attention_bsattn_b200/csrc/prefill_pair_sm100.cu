@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
   int b, hs[2], is[2], ns[2];
   const int32_t* cols = nullptr;
   int n;  // length of the shared K/V stream
+  int lenb = p.N;   // valid tokens of this CTA's sequence (key padding)
   if (!p.pair_tiles) {
     const int PH = p.Hq / 2;
     int i, bp;
@@ -135,6 +136,8 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
     hs[0] = 2 * (bp % PH);
     hs[1] = hs[0] + 1;
     is[0] = is[1] = i;
+    if (p.seq_lens) lenb = min(max(p.seq_lens[b], 0), p.N);
+    const int nkb = (lenb + BLK - 1) / BLK;   // key tiles holding valid keys
     // visit list of mask head 0, shared by both heads
     if (p.row_ptr) {
       const int32_t s0 = p.row_ptr[i];
@@ -143,9 +146,11 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
       n = s1 - s0;
       if (p.causal)
         while (n > 0 && cols[n - 1] > i) --n;
+      while (n > 0 && cols[n - 1] >= nkb) --n;
     } else {
-      n = p.causal ? i + 1 : p.nk;
+      n = min(p.causal ? i + 1 : p.nk, nkb);
     }
+    if (i * BLK >= lenb) n = 0;   // a query tile of padding visits nothing
     ns[0] = ns[1] = n;
   } else {
     const int NP = (p.nq + 1) / 2;
@@ -161,8 +166,10 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
     hs[0] = hs[1] = bh % p.Hq;
     is[0] = 2 * m;
     is[1] = 2 * m + 1;
-    ns[0] = p.causal ? is[0] + 1 : p.nk;
-    ns[1] = is[1] < p.nq ? (p.causal ? is[1] + 1 : p.nk) : 0;
+    if (p.seq_lens) lenb = min(max(p.seq_lens[b], 0), p.N);
+    const int nkb = (lenb + BLK - 1) / BLK;
+    ns[0] = is[0] * BLK < lenb ? min(p.causal ? is[0] + 1 : p.nk, nkb) : 0;
+    ns[1] = is[1] * BLK < lenb ? min(p.causal ? is[1] + 1 : p.nk, nkb) : 0;
     n = max(ns[0], ns[1]);
   }
   const int kvh = hs[0] / (p.Hq / p.Hkv);
@@ -395,7 +402,8 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
     // the tile index itself without one)
     const int du = p.reverse ? -1 : 1;
     const int u0 = p.reverse ? n - 1 - t_first : t_first;
-    const bool valid = r0 + row < p.N;
+    const bool valid = r0 + row < lenb;    // votes, and gets an output
+    const bool in_buf = r0 + row < p.N;    // written (padding rows as zeros)
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t s_col = 256 * e, o_col = 256 * e + 128;
     float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
@@ -415,12 +423,12 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
         tmem_ld32(lane_addr + s_col + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
       tmem_wait_ld();
       const int k0 = j * BLK;
-      if (k0 + BLK > p.N || (p.causal && j == i)) {
+      if (k0 + BLK > lenb || (p.causal && j == i)) {
         const int qpos = r0 + row;
 #pragma unroll
         for (int c = 0; c < BLK; ++c) {
           const int key = k0 + c;
-          if (key >= p.N || (p.causal && key > qpos)) r[c] = __float_as_uint(-INFINITY);
+          if (key >= lenb || (p.causal && key > qpos)) r[c] = __float_as_uint(-INFINITY);
         }
       }
       const float mx = row_max<BLK>(reinterpret_cast<const float*>(r));
@@ -522,7 +530,7 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
     if (ok) {
       const int64_t orow = ((int64_t)b * p.Hq + h) * p.N + r0 + row;
       __nv_bfloat16* dst = p.o + orow * D;
-      const bool have = kept > 0 && l > 0.f;
+      const bool have = valid && kept > 0 && l > 0.f;
       const float inv_l = have ? 1.f / l : 0.f;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
@@ -531,7 +539,7 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
           tmem_ld32(lane_addr + o_col + c0, ro);
           tmem_wait_ld();
         }
-        if (valid) {
+        if (in_buf) {
           uint32_t w[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
@@ -545,7 +553,7 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
             d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
-      if (valid && p.lse)
+      if (in_buf && p.lse)
         p.lse[orow] = have ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }

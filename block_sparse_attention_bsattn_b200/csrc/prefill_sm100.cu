@@ -119,6 +119,9 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
   }
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int kvh = h / (p.Hq / p.Hkv);
+  // valid tokens of this sequence (key padding) and the key tiles holding them
+  const int lenb = p.seq_lens ? min(max(p.seq_lens[b], 0), p.N) : p.N;
+  const int nkb = (lenb + BLK - 1) / BLK;
 
   // ---- visit list
   const int32_t* cols = nullptr;
@@ -131,9 +134,11 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
     n = s1 - s0;
     if (p.causal)
       while (n > 0 && cols[n - 1] > i) --n;
+    while (n > 0 && cols[n - 1] >= nkb) --n;
   } else {
-    n = p.causal ? i + 1 : p.nk;
+    n = min(p.causal ? i + 1 : p.nk, nkb);
   }
+  if (i * BLK >= lenb) n = 0;   // a query tile of padding visits nothing
   // key tile of visit step t (ascending, or descending on request)
   auto col_at = [&](int t) -> int {
     const int u = p.reverse ? n - 1 - t : t;
@@ -324,7 +329,8 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
     const int row = quarter * 32 + lane;    // query row inside the tile
     const int r0 = i * BLK;
     const bool in_tile = row < BLK;
-    const bool valid = in_tile && (r0 + row < p.N);
+    const bool valid = in_tile && (r0 + row < lenb);   // votes, and gets an output
+    const bool in_buf = in_tile && (r0 + row < p.N);   // written (padding rows as zeros)
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     float* xmax = reinterpret_cast<float*>(smem + C::XM_OFF);   // [2][2][128]
     float* lx = xmax + 2 * 2 * 128;                               // [2][128]
@@ -375,12 +381,12 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
         for (int c = 0; c < CW; ++c) s[c] = __uint_as_float(r[c]);
         // element masks: keys past the end, and keys after the query (causal)
         const int k0 = j * BLK + half * CW;
-        if (j * BLK + BLK > p.N || (p.causal && j == i)) {
+        if (j * BLK + BLK > lenb || (p.causal && j == i)) {
           const int qpos = r0 + row;
 #pragma unroll
           for (int c = 0; c < CW; ++c) {
             const int key = k0 + c;
-            if (key >= p.N || (p.causal && key > qpos)) s[c] = -INFINITY;
+            if (key >= lenb || (p.causal && key > qpos)) s[c] = -INFINITY;
           }
         }
         mh = row_max<CW>(s);
@@ -503,7 +509,7 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
       const float lt = lx[row] + lx[128 + row];
       const int64_t orow = ((int64_t)b * p.Hq + h) * p.N + r0 + row;
       __nv_bfloat16* dst = p.o + orow * D + half * OW;
-      const bool have = kept > 0 && lt > 0.f;
+      const bool have = valid && kept > 0 && lt > 0.f;
       const float inv_l = have ? 1.f / lt : 0.f;
 #pragma unroll
       for (int c0 = 0; c0 < OW; c0 += 32) {
@@ -512,7 +518,7 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
           tmem_ld32(lane_addr + C::O_COL + half * OW + c0, r);
           tmem_wait_ld();
         }
-        if (valid) {
+        if (in_buf) {
           uint32_t w[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
@@ -526,7 +532,7 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
             d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
-      if (valid && half == 0 && p.lse)
+      if (in_buf && half == 0 && p.lse)
         p.lse[orow] = have ? (m_ref + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
     }
   }

@@ -88,9 +88,37 @@ def table4(args):
     return rows
 
 
+def varlen(args):
+    """Causal BLASST prefill over a batch padded to N = 16384 with valid
+    lengths 16384, 12288, 8192 and 4096 (32 query / 8 KV heads), against the
+    same batch without lengths (every sequence full)."""
+    B, H, Hkv, N = 4, 32, 8, 16384
+    q, k, v = inputs.blasst_prefill_qkv(B, H, Hkv, N, 128, "cuda", 5150)
+    lens = torch.tensor([16384, 12288, 8192, 4096], dtype=torch.int32, device="cuda")
+    o = torch.empty_like(q)
+    nq = N // 128
+    rows = []
+    for name, sl in (("padded_full", None), ("varlen", lens)):
+        lam = inputs.lambda_for(args.a, N)
+        st = torch.zeros(B, H, nq, nq, dtype=torch.uint8, device="cuda")
+        ops.bsattn_fwd_prefill(q, k, v, 128, None, True, lam, o=o, tile_status=st, want_lse=False,
+                               seq_lens=sl)
+        torch.cuda.synchronize()
+        vis, exe = int((st > 0).sum()), int((st == 2).sum())
+        fn = lambda: ops.bsattn_fwd_prefill(q, k, v, 128, None, True, lam, o=o, want_lse=False,
+                                            seq_lens=sl)
+        for _ in range(args.warmup):
+            fn()
+        ms = _time(fn, args.iters)
+        rows.append({"case": name, "a": args.a, "visited": vis, "executed": exe, "ms": ms,
+                     "tflops": TILE * (vis + exe) / ms / 1e9})
+    return rows
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=("prefill", "decode", "videodit", "mmdit", "table4"))
+    ap.add_argument("what", choices=("prefill", "decode", "videodit", "mmdit", "table4",
+                                     "varlen"))
     ap.add_argument("--heads", type=int, default=8, help="query heads (prefill/videodit/mmdit)")
     ap.add_argument("--n", type=int, default=32768, help="sequence length (prefill)")
     ap.add_argument("--batch", type=int, default=64, help="batch (decode)")
@@ -142,6 +170,8 @@ def main():
         out.update(heads=args.heads, n=w.N, d=w.d, tiles=tiles, ms=ms, tflops=flops / ms / 1e9)
     elif args.what == "table4":
         out["rows"] = table4(args)
+    elif args.what == "varlen":
+        out["rows"] = varlen(args)
     else:
         B, Hq, Hkv, L, d = args.batch, 32, args.hkv, args.l, 128
         ns = args.splits

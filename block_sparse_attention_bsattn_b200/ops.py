@@ -43,7 +43,7 @@ _lib.bsattn_fwd_prefill.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, 
                                     _P, _P, _P, _I, _P, _P, _P]
 _lib.bsattn_fwd_prefill.restype = _I
 _lib.bsattn_fwd_prefill_ex.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F,
-                                       _P, _P, _P, _I, _P, ctypes.c_uint, _P, _P]
+                                       _P, _P, _P, _I, _P, _P, ctypes.c_uint, _P, _P]
 _lib.bsattn_fwd_prefill_ex.restype = _I
 _lib.bsattn_decode_workspace_size.argtypes = [_I, _I, _I, _I]
 _lib.bsattn_decode_workspace_size.restype = _SZ
@@ -51,7 +51,7 @@ _lib.bsattn_fwd_decode.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _
                                    _P, _SZ, _P, _P, _P]
 _lib.bsattn_fwd_decode.restype = _I
 _lib.bsattn_fwd_decode_ex.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F,
-                                      _I, _P, _SZ, _P, ctypes.c_uint, _P, _P]
+                                      _I, _P, _SZ, _P, _P, ctypes.c_uint, _P, _P]
 _lib.bsattn_fwd_decode_ex.restype = _I
 _lib.bsattn_fwd_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I,
                                            _F, _I, _P, _P, _P]
@@ -153,11 +153,13 @@ def bsattn_fwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
                        want_lse: bool = True, tile_status: Optional[torch.Tensor] = None,
                        status: Optional[torch.Tensor] = None,
                        row_order: Optional[torch.Tensor] = None, stream=None,
-                       reverse: bool = False, skip_v: bool = False):
+                       reverse: bool = False, skip_v: bool = False,
+                       seq_lens: Optional[torch.Tensor] = None):
     """q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 -> (o [B,Hq,N,d] bf16, lse [B,Hq,N] fp32 or None).
     reverse: visit each row's key tiles in descending order; skip_v: load V
     only for executed tiles (bsattn_fwd_prefill_ex with BSATTN_PREFILL_REVERSE
-    / BSATTN_PREFILL_SKIP_V)."""
+    / BSATTN_PREFILL_SKIP_V); seq_lens: int32 [B] on the device, valid tokens
+    per sequence (key padding)."""
     _check(q, "q", torch.bfloat16, 4)
     _check(k, "k", torch.bfloat16, 4)
     _check(v, "v", torch.bfloat16, 4)
@@ -175,8 +177,13 @@ def bsattn_fwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
             float(scale), int(causal), float(lam), _ptr(row_ptr), _ptr(col_idx), _ptr(row_order),
             int(mask_heads), _ptr(tile_status))
     flags = (PREFILL_REVERSE if reverse else 0) | (PREFILL_SKIP_V if skip_v else 0)
-    if flags:
-        rc = _lib.bsattn_fwd_prefill_ex(*args, flags, _ptr(status), _stream(stream))
+    if seq_lens is not None:
+        _check(seq_lens, "seq_lens", torch.int32, 1)
+        if seq_lens.numel() != B:
+            raise ValueError("seq_lens must hold B lengths")
+    if flags or seq_lens is not None:
+        rc = _lib.bsattn_fwd_prefill_ex(*args, _ptr(seq_lens), flags, _ptr(status),
+                                        _stream(stream))
     else:
         rc = _lib.bsattn_fwd_prefill(*args, _ptr(status), _stream(stream))
     if rc:
@@ -194,10 +201,11 @@ def bsattn_fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: 
                       want_lse: bool = True, workspace: Optional[torch.Tensor] = None,
                       tile_status: Optional[torch.Tensor] = None,
                       status: Optional[torch.Tensor] = None, stream=None,
-                      sink_seed: bool = False):
+                      sink_seed: bool = False, seq_lens: Optional[torch.Tensor] = None):
     """q [B,Hq,d], k/v [B,Hkv,L,d] bf16 -> (o [B,Hq,d] bf16, lse [B,Hq] fp32 or None).
     sink_seed: splits after the first start their running max from key tile
-    0's row max (calls bsattn_fwd_decode_ex with BSATTN_DECODE_SINK_SEED)."""
+    0's row max (calls bsattn_fwd_decode_ex with BSATTN_DECODE_SINK_SEED);
+    seq_lens: int32 [B] on the device, cache length per sequence."""
     _check(q, "q", torch.bfloat16, 3)
     _check(k, "k", torch.bfloat16, 4)
     _check(v, "v", torch.bfloat16, 4)
@@ -217,8 +225,13 @@ def bsattn_fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: 
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, L, d, int(block),
             float(scale), 0, float(lam), int(num_splits), _ptr(workspace),
             workspace.numel() * workspace.element_size(), _ptr(tile_status))
-    if sink_seed:
-        rc = _lib.bsattn_fwd_decode_ex(*args, DECODE_SINK_SEED, _ptr(status), _stream(stream))
+    if seq_lens is not None:
+        _check(seq_lens, "seq_lens", torch.int32, 1)
+        if seq_lens.numel() != B:
+            raise ValueError("seq_lens must hold B lengths")
+    if sink_seed or seq_lens is not None:
+        rc = _lib.bsattn_fwd_decode_ex(*args, _ptr(seq_lens), DECODE_SINK_SEED if sink_seed else 0,
+                                       _ptr(status), _stream(stream))
     else:
         rc = _lib.bsattn_fwd_decode(*args, _ptr(status), _stream(stream))
     if rc:

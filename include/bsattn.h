@@ -162,6 +162,14 @@ int bsattn_fwd_prefill(const void *q, const void *k, const void *v, void *o, flo
  * and tile_status -- are those of the reversed order; with lambda = 0 only
  * the summation order changes.
  *
+ * d_seq_lens: NULL, or int32 [B] in device memory: sequence b holds
+ * d_seq_lens[b] valid tokens (values are clamped to [0, N]), the rest of its
+ * N positions are padding ("块稀疏Attention实战" section 5.2: pad a batch to its
+ * longest sequence and mask the padding keys).  Keys at or past the length
+ * take no part, key tiles wholly past it are not visited, and query rows past
+ * it are padding: they do not vote and get O = 0 and LSE = -inf.  Every
+ * sequence's result equals that of the sequence alone at its own length.
+ *
  * BSATTN_PREFILL_SKIP_V: a V tile is loaded only when some query tile that
  * shares it executes it, instead of for every visited tile.  Results are
  * unchanged.  The BLASST page's prefill kernel loads every V tile (section
@@ -173,8 +181,8 @@ int bsattn_fwd_prefill_ex(const void *q, const void *k, const void *v, void *o, 
                           int B, int Hq, int Hkv, int N, int d, int block, float scale,
                           int causal, float lambda, const int32_t *row_ptr,
                           const int32_t *col_idx, const int32_t *row_order, int mask_heads,
-                          uint8_t *tile_status, unsigned flags, int32_t *d_status,
-                          cudaStream_t stream);
+                          uint8_t *tile_status, const int32_t *d_seq_lens, unsigned flags,
+                          int32_t *d_status, cudaStream_t stream);
 
 /*
  * bsattn_decode_workspace_size -- bytes of scratch bsattn_fwd_decode needs:
@@ -227,12 +235,18 @@ int bsattn_fwd_decode(const void *q, const void *k, const void *v, void *o, floa
  * and test the rest against its own, smaller maxima.  (The pages define no
  * split-KV; this variant keeps their skip rule and only changes the starting
  * value of each split's running max.)
+ *
+ * d_seq_lens: NULL, or int32 [B] in device memory: cache b holds d_seq_lens[b]
+ * valid tokens (clamped to [0, L]); keys past it take no part, and the
+ * num_splits splits cut that cache's own ceil(len / block) tiles, so every
+ * sequence's result equals that of its cache alone.  A zero length gives
+ * O = 0 and LSE = -inf.
  */
 int bsattn_fwd_decode_ex(const void *q, const void *k, const void *v, void *o, float *lse,
                          int B, int Hq, int Hkv, int L, int d, int block, float scale, int causal,
                          float lambda, int num_splits, void *workspace, size_t workspace_bytes,
-                         uint8_t *tile_status, unsigned flags, int32_t *d_status,
-                         cudaStream_t stream);
+                         uint8_t *tile_status, const int32_t *d_seq_lens, unsigned flags,
+                         int32_t *d_status, cudaStream_t stream);
 
 /*
  * bsattn_fwd_decode_noalloc -- bsattn_fwd_decode for callers that cannot

@@ -98,20 +98,20 @@ def test_option_bits_validation(lib):
     """The _ex entry points reject unknown option bits before anything runs."""
     U = ctypes.c_uint
     lib.bsattn_fwd_prefill_ex.argtypes = [P, P, P, P, P] + [ctypes.c_int] * 6 + [
-        ctypes.c_float, ctypes.c_int, ctypes.c_float, P, P, P, ctypes.c_int, P, U, P, P]
+        ctypes.c_float, ctypes.c_int, ctypes.c_float, P, P, P, ctypes.c_int, P, P, U, P, P]
     lib.bsattn_fwd_decode_ex.argtypes = [P, P, P, P, P] + [ctypes.c_int] * 6 + [
-        ctypes.c_float, ctypes.c_int, ctypes.c_float, ctypes.c_int, P, ctypes.c_size_t, P, U,
+        ctypes.c_float, ctypes.c_int, ctypes.c_float, ctypes.c_int, P, ctypes.c_size_t, P, P, U,
         P, P]
 
     def pre(flags, q=0x1000):
         return lib.bsattn_fwd_prefill_ex(P(q) if q else None, P(0x2000), P(0x3000), P(0x4000),
                                          None, 1, 2, 2, 256, 128, 128, 0.1, 0, 0.0, None, None,
-                                         None, 1, None, flags, None, None)
+                                         None, 1, None, None, flags, None, None)
 
     def dec(flags, q=0x1000):
         return lib.bsattn_fwd_decode_ex(P(q) if q else None, P(0x2000), P(0x3000), P(0x4000),
                                         None, 2, 8, 2, 1000, 128, 128, 0.1, 0, 0.0, 4, P(0x9000),
-                                        1 << 30, None, flags, None, None)
+                                        1 << 30, None, None, flags, None, None)
     assert pre(0x4) == -1 and pre(0x80000000) == -1
     assert pre(0x1, q=0) == -1
     assert dec(0x2) == -1 and dec(0x1, q=0) == -1

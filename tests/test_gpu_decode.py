@@ -95,6 +95,38 @@ def test_sink_seed_with_empty_splits():
     _check(q, k, v, 128, 8, 1 / math.sqrt(128), 1e-2, what="seeded empty splits", sink_seed=True)
 
 
+@pytest.mark.parametrize("d,block,g", [(128, 128, 4), (64, 128, 8), (128, 64, 4), (64, 64, 2)])
+@pytest.mark.parametrize("sink_seed", [False, True])
+def test_varlen_cache_lengths(d, block, g, sink_seed):
+    """Per-sequence cache lengths: both decode kernels against the oracle's
+    problems at their own lengths (splits cut each cache's own tiles)."""
+    ops = _ops()
+    B, Hkv, L, splits = 5, 2, 19 * block + 11, 4
+    lens = [L, 7 * block + 3, block, 1, 0]
+    q, k, v = inputs.blasst_decode_qkv(B, Hkv * g, Hkv, L, d, "cpu", 61 + g + block)
+    lam = 1e-2
+    T = -(-L // block)
+    st = torch.zeros(B, Hkv, T, dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    o, lse = ops.bsattn_fwd_decode(q.cuda(), k.cuda(), v.cuda(), block, splits, 1 / math.sqrt(d),
+                                   lam, tile_status=st, status=status, sink_seed=sink_seed,
+                                   seq_lens=sl)
+    torch.cuda.synchronize()
+    assert status.item() == 0, ops.bsattn_status_string(status.item())
+    pairs = [(b, h) for b in range(B) for h in range(Hkv)]
+    qs, ks, vs = oracle.decode_problems(q, k, v, pairs)
+    ref = oracle.decode(qs.cpu(), ks.cpu(), vs.cpu(), block, 1 / math.sqrt(d), lam, splits,
+                        sink_seed=sink_seed, lens=[lens[b] for b, _ in pairs])
+    o_c, lse_c, st_c = o.float().cpu().numpy(), lse.cpu().numpy(), st.cpu().numpy()
+    for p_, (b, kvh) in enumerate(pairs):
+        rows = slice(kvh * g, (kvh + 1) * g)
+        compare_outputs(o_c[b, rows], ref["o"][p_], lse_c[b, rows], ref["lse"][p_],
+                        f"varlen decode pair {(b, kvh)}")
+        compare_status(st_c[b, kvh], ref["status"][p_], ref["margin"][p_], "varlen decode")
+    assert (o_c[4] == 0).all() and np.isneginf(lse_c[4]).all()   # an empty cache
+
+
 def test_more_splits_than_tiles():
     q, k, v = inputs.blasst_decode_qkv(1, 4, 1, 300, 128, "cpu", 9)
     _check(q, k, v, 128, 8, 1 / math.sqrt(128), 1e-2, what="empty splits")

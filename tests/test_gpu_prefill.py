@@ -209,6 +209,52 @@ def test_skip_v_dense_and_full_size_sampled():
         compare_status(st_c[b, h, i], ref["status"][b, h, i], ref["margin"][b, h, i])
 
 
+@pytest.mark.parametrize("hq,hkv,block,causal,masked", [
+    (4, 2, 128, True, False),    # two heads of one KV head per CTA
+    (2, 2, 128, True, False),    # two consecutive query tiles per CTA
+    (1, 1, 128, False, False),
+    (2, 1, 64, True, False),     # one query tile per CTA
+    (4, 2, 128, False, True),    # shared mask: two heads per CTA, CSR visit lists
+    (4, 4, 64, True, True),      # per-head masks
+])
+@pytest.mark.parametrize("reverse", [False, True])
+def test_varlen_key_padding(hq, hkv, block, causal, masked, reverse):
+    """Per-sequence valid lengths (key padding): every kernel against the
+    oracle's padded batch, lengths 0, partial tiles, tile multiples and full."""
+    B, N = 5, 6 * block + 29
+    lens = [N, 3 * block + 5, block, 0, 17]
+    q, k, v = inputs.blasst_prefill_qkv(B, hq, hkv, N, 128, "cpu", 91 + block)
+    ops = _ops()
+    rp = ci = None
+    mh = 1
+    mask = None
+    nb = -(-N // block)
+    if masked:
+        rng = np.random.default_rng(11)
+        heads = 1 if hq != hkv else hq
+        mask = (rng.random((heads, nb, nb)) < 0.6).astype(np.uint8)
+        mask[:, np.arange(nb), np.arange(nb)] = 1
+        m = torch.as_tensor(mask).cuda().contiguous()
+        rp, ci, _ = ops.bsattn_build_index(m, block, block, causal)
+        mh = heads
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    st = torch.zeros(B, hq, nb, nb, dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lam = 0.02
+    o, lse = ops.bsattn_fwd_prefill(q.cuda(), k.cuda(), v.cuda(), block, 1 / math.sqrt(128),
+                                    causal, lam, rp, ci, mh, tile_status=st, status=status,
+                                    reverse=reverse, seq_lens=sl)
+    torch.cuda.synchronize()
+    assert status.item() == 0, ops.bsattn_status_string(status.item())
+    ref = oracle.prefill(q, k, v, block, 1 / math.sqrt(128), causal, lam, mask=mask,
+                         reverse=reverse, seq_lens=lens)
+    compare_outputs(o, ref["o"], lse, ref["lse"], f"varlen h{hq}/{hkv} b{block} rev{reverse}")
+    compare_status(st, ref["status"], ref["margin"], "varlen")
+    for b, L in enumerate(lens):     # padding rows: exactly zero and -inf
+        assert (o[b, :, L:].float() == 0).all()
+        assert torch.isneginf(lse[b, :, L:]).all()
+
+
 def test_short_sequence_single_partial_tile():
     q, k, v = inputs.normal_qkv(1, 2, 2, 50, 128, "cpu", 3)
     w = inputs.Workload("short", 1, 2, 2, 50, 128, 128, True, "prefill", 1 / math.sqrt(128), None,
