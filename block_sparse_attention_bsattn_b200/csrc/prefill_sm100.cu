@@ -145,16 +145,10 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
     return cols ? cols[u] : u;
   };
 
-  // debug trace: slot 16 + CTA = stage reached; CTA 0 also records per-role
-  // progress, and an SM-clock timeline of its first tiles from slot 1024 on
-  // (8 slots per tile: BMM1 issued, P seen by the MMA warp, BMM2 issued, S seen
-  // by the softmax, votes agreed, P handed back)
+  // debug trace: slot 16 + CTA = stage reached (set-up, pipeline, teardown);
+  // CTA 0 also marks each warp's exit.  Nothing is recorded per tile: markers
+  // on the MMA warp's path measured 5% slower in the two-tile kernel.
   const bool tr0 = blockIdx.x == 0;
-  auto tl_mark = [&](int t, int k) {   // plain store: no fence, read after the kernel
-    if (tr0 && p.trace && 1024 + t * 8 + k < p.trace_n) {
-      p.trace[1024 + t * 8 + k] = (int32_t)clock64();
-    }
-  };
   if (threadIdx.x == 0) trace_mark(p.trace, p.trace_n, 16 + blockIdx.x, 1);
 
   // ---- setup
@@ -218,9 +212,7 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
           tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
                       hf * 64, j * BLK, b * p.Hkv + kvh);
         ++issued_v;
-        if (tr0) trace_mark(p.trace, p.trace_n, 1, t + 1);
       }
-      if (tr0) trace_mark(p.trace, p.trace_n, 1, 100000 + issued_k);
       if (*abort) {
         // let every copy this thread started land before the CTA can exit
         for (int t = (issued_k > C::KST ? issued_k - C::KST : 0); t < issued_k; ++t)
@@ -275,7 +267,6 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
         }
         mma_commit(&bars->s_full[t & 1]);
         mma_commit(&bars->k_empty[ks]);
-        tl_mark(t, 0);
         return true;
       };
       if (ok) ok = issue_bmm1(0);
@@ -285,7 +276,6 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
         const int sb = t & 1;
         if (!mbar_wait(&bars->p_ready[sb], (t >> 1) & 1, abort, lim)) break;
         tc_fence_after();
-        tl_mark(t, 1);
         const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[sb]);
         // V ring position: every visited tile's, or (V skipping) the kept ones'
         const int vi = SKIPV ? kept : t;
@@ -303,18 +293,14 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
           }
           mma_commit(&bars->o_done);
           mma_commit(&bars->v_empty[vs]);
-          tl_mark(t, 2);
           ++kept;
         } else if (!SKIPV) {
           mbar_arrive(&bars->v_empty[vs]);
         }
-        if (tr0) trace_mark(p.trace, p.trace_n, 2, t + 1);
       }
-      if (tr0) trace_mark(p.trace, p.trace_n, 2, 100000 + kept);
       // all tcgen05 work issued by this thread must finish before TMEM is freed
       mma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0, lim);
-      if (tr0) trace_mark(p.trace, p.trace_n, 3, 1);
     }
   } else {
     // ======================================================== softmax warps
@@ -367,7 +353,6 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
         break;
       }
       tc_fence_after();
-      if (sw == 0 && lane == 0) tl_mark(t, 3);
       float s[CW];
       float mh = -INFINITY;
       if (in_tile) {
@@ -405,7 +390,6 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
         ok = false;
         break;
       }
-      if (sw == 0 && lane == 0) tl_mark(t, 4);
       int skip = 0;
       if (p.use_skip) {
         volatile int* vv = bars->vote[t & 1];
@@ -487,8 +471,6 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready[sb]);
-      if (sw == 0 && lane == 0) tl_mark(t, 5);
-      if (tr0 && lane == 0) trace_mark(p.trace, p.trace_n, 4 + (sw & 3), t + 1);
     }
 
     // ---- epilogue: row sums of both halves, O / l -> bf16, LSE.  tcgen05.ld

@@ -78,7 +78,8 @@ int bsattn_debug_set(long long wait_limit_ns, int inject_stall);
  * the prefill and decode kernels record progress there, readable while a
  * kernel is still running: slot 16 + CTA index holds the stage a CTA reached
  * (1 entered, 2 set up, 3 finished, 4 tensor memory freed; 13/14 the same
- * after a timed-out wait), slots 1..11 the per-role progress of CTA 0.  n = 0
+ * after a timed-out wait), slots 8..17 the warps of CTA 0 that have left
+ * their role's loop (one-query-tile prefill kernel).  n = 0
  * frees the buffer and turns tracing off.  Negative n or a NULL host_view
  * with n > 0 give BSATTN_ERR_INVALID_ARG.
  */
