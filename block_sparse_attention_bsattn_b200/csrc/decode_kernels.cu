@@ -13,7 +13,7 @@
 //   Per visited tile t:
 //     QK     each key is owned by 32/KPW lanes of a warp (KPW keys per warp),
 //            each lane dots a slice of d for all G rows; lanes combine with
-//            xor-shuffles; masks keys past L.
+//            xor-shuffles; masks keys past the cache length.
 //     max    warp max -> shared memory -> every thread forms the tile max
 //            per row, the skip decision (all G rows below running max +
 //            log2(lambda)) and the new running max, identically.
@@ -22,7 +22,8 @@
 //            the next tiles' K streaming and scores.  The exponent shift is
 //            lazy: it only moves when the running max exceeds it by more than
 //            TAU, and then the partial O and row sums are rescaled first.
-//   The split writes its unnormalised O (fp32), shift and row sum.
+//   The split writes its unnormalised O (fp32), shift and row sum.  Options
+//   as in the tensor-core kernel: sink-seeded splits, per-sequence lengths.
 // decode_combine_kernel: one CTA per (batch, query head): log-sum-exp merge of
 //   the splits into bf16 O and fp32 LSE.
 #include <cmath>

@@ -30,6 +30,11 @@
 // The exponent shift is lazy: it moves only when the running max exceeds it by
 // more than TAU (base 2); O^T and the row sums are then rescaled after every
 // earlier P.V has completed.  Every wait is bounded in time.
+// The softmax warps' per-column loops run over NC columns, g rounded up to a
+// power of two and fixed at compile time (one instance per NC), and the
+// per-warp tile max is a butterfly reduce-scatter.  Options: sink-seeded
+// splits (an extra first step scores key tile 0 to start the running max)
+// and per-sequence cache lengths (the splits cut each cache's own tiles).
 #include <cmath>
 #include <cstdint>
 #include <cuda.h>

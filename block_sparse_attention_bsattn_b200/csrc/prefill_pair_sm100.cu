@@ -4,30 +4,32 @@
 //               (GQA group of even size, one visit list for the group);
 //   tiles mode  two consecutive query tiles of one head when no block mask is
 //               given (every key tile, or the causal prefix, which differs by
-//               the diagonal tile only): slot e visits stream tiles t < n_e.
+//               the diagonal tile only).  Each slot takes part in a range of
+//               the stream's steps: a prefix in ascending visit order, a
+//               suffix in descending order.
 //
 // Same method as prefill_sm100.cu ("BLASST: Dynamic Blocked Attention Sparsity
 // via Softmax Thresholding", Algorithm 1 and section 4.1; "块稀疏Attention实战"
-// section 3.3): per query tile, visited key tiles in ascending order, S = Q K^T
-// for each, the row max, the skip test against the running max, and for kept
-// tiles P = exp(S - m), the row sums and O += P V.  The two heads' skip
-// decisions are independent.
+// section 3.3): per query tile, visited key tiles in order, S = Q K^T for each,
+// the row max, the skip test against the running max, and for kept tiles
+// P = exp(S - m), the row sums and O += P V.  The two slots' skip decisions
+// are independent.  Optional: descending visit order, per-sequence lengths
+// (key padding), V loads only for kept tiles.
 //
 // 10 warps (11 with V skipping):
-//   warp 0      TMA producer: Q of both heads, then K_j (3-stage ring) and V_j
+//   warp 0      TMA producer: Q of both slots, then K_j (3-stage ring) and V_j
 //               (2-stage ring)
+//   warp 1      TMEM owner, MMA issuer.  The two query tiles ping-pong: after
+//               slot A's P is ready its BMM2 and its next BMM1 are issued, then
+//               slot B's, so the tensor core works on one slot while the other
+//               slot's softmax runs.
+//   warps 2..5  softmax of slot A, warps 6..9 softmax of slot B: one thread per
+//               query row (TMEM lane), vote across the four warps of the slot.
 //   warp 10     with V skipping only: the V producer.  The section on the
 //               prefill kernel keeps every V load (the decision comes too late
 //               to hide a conditional load's latency); as an option, a slot's
 //               softmax sends each decision through a queue and V_j is loaded
-//               only when some slot keeps tile j, which halves the bytes a
-//               skipped step pulls from L2.
-//   warp 1      TMEM owner, MMA issuer.  The two query tiles ping-pong: after
-//               head A's P is ready its BMM2 and its next BMM1 are issued, then
-//               head B's, so the tensor core works on one head while the other
-//               head's softmax runs.
-//   warps 2..5  softmax of head A, warps 6..9 softmax of head B: one thread per
-//               query row (TMEM lane), vote across the four warps of the head.
+//               only when some slot keeps tile j.
 // TMEM: S_A [0,128)  O_A [128,256)  S_B [256,384)  O_B [384,512).
 // BMM1: A = Q (smem, K-major, 128B swizzle), B = K tile (smem, K-major).
 // BMM2: A = P (TMEM, bf16 over S), B = V tile (smem, MN-major).

@@ -1,32 +1,37 @@
 // Block-sparse attention prefill for sm_100a: tcgen05 tensor-core MMAs with
 // TMEM accumulators, TMA-staged tiles, warp-specialised roles, and the BLASST
-// skip test inside the online softmax.
+// skip test inside the online softmax.  Serves the cases the two-tile kernel
+// does not: 64-token tiles, per-head block masks, odd GQA groups with a mask.
 //
 // What it computes ("BLASST: Dynamic Blocked Attention Sparsity via Softmax
 // Thresholding", Algorithm 1 and section 4.1; "块稀疏Attention实战" section
 // 3.3): for each query tile, the key tiles of its visit list are processed in
-// ascending order; every visited tile gets S = Q K^T (BMM1), its row max, and
-// the skip test against the running max; a kept tile then gets P = exp(S - m)
-// (CUDA cores), the row sums, and O += P V (BMM2).  A skipped tile costs one
-// BMM1 and a row max.
+// order (ascending, or descending on request); every visited tile gets
+// S = Q K^T (BMM1), its row max, and the skip test against the running max; a
+// kept tile then gets P = exp(S - m) (CUDA cores), the row sums, and O += P V
+// (BMM2).  A skipped tile costs one BMM1 and a row max.  Optional per-sequence
+// lengths mask padding keys and rows.
 //
-// One CTA = one (batch, head, query tile) work item; 10 warps:
-//   warp 0      TMA producer: Q once, then K_j and V_j of every visited tile
-//               into 3-stage rings (V is loaded for every visited tile, as the
-//               BLASST prefill kernel does -- the load is not on the critical
-//               path of a compute-bound kernel);
+// One CTA = one (batch, head, query tile) work item; 10 warps (11 with V
+// skipping):
+//   warp 0      TMA producer: K_j and V_j of every visited tile into 3-stage
+//               rings (V is loaded for every visited tile, as the BLASST
+//               prefill kernel does, unless V skipping is requested: then
+//               warp 10 loads V for kept tiles only, from a decision queue);
 //   warp 1      TMEM owner and MMA issuer (one elected lane): BMM1 of tile
 //               t + 1 is issued before waiting for the softmax of tile t, so
 //               the tensor core works while the softmax warps do;
 //   warps 2..9  softmax, two warpgroups: each query row (TMEM lane) is shared
 //               by one thread of each warpgroup, which own the low and the
 //               high half of the score columns (and of the output columns).
-//               Per tile one shared-memory round exchanges the half-row maxima
+//               They first write the query tile into TMEM (bf16 pairs).  Per
+//               tile one shared-memory round exchanges the half-row maxima
 //               and the warp votes (__all_sync per warp; a row passes iff both
 //               halves pass); P = exp2 goes back to TMEM as bf16 over the
 //               tile's S columns; lazy rescale of O; the epilogue.
-// TMEM columns: S double buffer at [0,128) and [128,256), O at [256, 256+d).
-// BMM1: A = Q (smem, K-major, 128B swizzle), B = K tile (smem, K-major).
+// TMEM columns: S double buffer at [0,128) and [128,256), O at [256, 256+d),
+// Q at [384, 384 + d/2).
+// BMM1: A = Q (TMEM), B = K tile (smem, K-major, 128B swizzle).
 // BMM2: A = P (TMEM), B = V tile (smem, MN-major, 128B swizzle).
 // The query tile always occupies 128 MMA rows; with 64-token tiles rows
 // 64..127 carry no data and their outputs are never read.
