@@ -16,16 +16,17 @@
 // are independent.  Optional: descending visit order, per-sequence lengths
 // (key padding), V loads only for kept tiles.
 //
-// 10 warps (11 with V skipping):
+// 12 warps in three warpgroups; warpgroup 0 hands registers to the two
+// softmax warpgroups (setmaxnreg: 56 / 224 per thread):
 //   warp 0      TMA producer: Q of both slots, then K_j (3-stage ring) and V_j
 //               (2-stage ring)
 //   warp 1      TMEM owner, MMA issuer.  The two query tiles ping-pong: after
 //               slot A's P is ready its BMM2 and its next BMM1 are issued, then
 //               slot B's, so the tensor core works on one slot while the other
 //               slot's softmax runs.
-//   warps 2..5  softmax of slot A, warps 6..9 softmax of slot B: one thread per
-//               query row (TMEM lane), vote across the four warps of the slot.
-//   warp 10     with V skipping only: the V producer.  The section on the
+//   warps 4..7  softmax of slot A, warps 8..11 softmax of slot B: one thread
+//               per query row (TMEM lane), vote across the four warps of the slot.
+//   warp 2      with V skipping only: the V producer (warp 3 idles).  The section on the
 //               prefill kernel keeps every V load (the decision comes too late
 //               to hide a conditional load's latency); as an option, a slot's
 //               softmax sends each decision through a queue and V_j is loaded
@@ -69,6 +70,10 @@ struct PairCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr float TAU = 8.0f;
   static constexpr int DQ = 4;                          // decision queue (V skipping)
+  static constexpr int THREADS = 384;                   // 3 warpgroups
+  static constexpr int REG_LAUNCH = 168;                // 65536 / 384, rounded down to 8
+  static constexpr int REG_LOW = 56;                    // warpgroup 0 after the split
+  static constexpr int REG_HIGH = 224;                  // softmax warpgroups after the split
 };
 
 struct PairBarriers {
@@ -89,7 +94,7 @@ struct PairBarriers {
 };
 
 template <int D, bool SKIPV>
-__global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
+__global__ void __launch_bounds__(384, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -222,342 +227,356 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const uint64_t lim = p.wait_limit_ns;
-
-  if (warp == 0) {
-    // ======================================================== TMA producer
-    if (lane == 0 && n > 0) {
-      prefetch_tensormap(&tmQ);
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
-      if (!p.debug_stall) {
-        mbar_arrive_expect_tx(&bars->q_full, 2 * C::HALVES * BLK * 128);
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
+  // register split: warpgroup 0 (producers, MMA) gives registers to the two
+  // softmax warpgroups.  128 * REG_LOW + 256 * REG_HIGH equals the 384 * 168
+  // the block is launched with (the launcher checks the kernel's count).
+  if (warp < 4) {
+    setmaxnreg_dec<C::REG_LOW>();
+    if (warp == 0) {
+      // ======================================================== TMA producer
+      if (lane == 0 && n > 0) {
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        if (!p.debug_stall) {
+          mbar_arrive_expect_tx(&bars->q_full, 2 * C::HALVES * BLK * 128);
+  #pragma unroll
+          for (int e = 0; e < 2; ++e)
+            for (int hf = 0; hf < C::HALVES; ++hf)
+              tma_load_3d(q_smem + e * C::Q_BYTES + hf * C::Q_HALF, &tmQ, &bars->q_full, hf * 64,
+                          is[e] * BLK, b * p.Hq + hs[e]);
+        }
+        int issued_k = 0, issued_v = 0;
+        for (int t = 0; t < n; ++t) {
+          const int j = col_at(t);
+          const int ks = t % C::KST;
+          if (!mbar_wait(&bars->k_empty[ks], ((t / C::KST) & 1) ^ 1, abort, lim)) break;
+          mbar_arrive_expect_tx(&bars->k_full[ks], C::T_BYTES);
           for (int hf = 0; hf < C::HALVES; ++hf)
-            tma_load_3d(q_smem + e * C::Q_BYTES + hf * C::Q_HALF, &tmQ, &bars->q_full, hf * 64,
-                        is[e] * BLK, b * p.Hq + hs[e]);
-      }
-      int issued_k = 0, issued_v = 0;
-      for (int t = 0; t < n; ++t) {
-        const int j = col_at(t);
-        const int ks = t % C::KST;
-        if (!mbar_wait(&bars->k_empty[ks], ((t / C::KST) & 1) ^ 1, abort, lim)) break;
-        mbar_arrive_expect_tx(&bars->k_full[ks], C::T_BYTES);
-        for (int hf = 0; hf < C::HALVES; ++hf)
-          tma_load_3d(k_smem + ks * C::T_BYTES + hf * C::T_HALF, &tmK, &bars->k_full[ks],
-                      hf * 64, j * BLK, b * p.Hkv + kvh);
-        ++issued_k;
-        if (SKIPV) continue;   // warp 10 loads V
-        const int vs = t % C::VST;
-        if (!mbar_wait(&bars->v_empty[vs], ((t / C::VST) & 1) ^ 1, abort, lim)) break;
-        mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
-        for (int hf = 0; hf < C::HALVES; ++hf)
-          tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
-                      hf * 64, j * BLK, b * p.Hkv + kvh);
-        ++issued_v;
-      }
-      if (*abort) {
-        for (int t = (issued_k > C::KST ? issued_k - C::KST : 0); t < issued_k; ++t)
-          mbar_wait_drain(&bars->k_full[t % C::KST], (t / C::KST) & 1, lim);
-        for (int t = (issued_v > C::VST ? issued_v - C::VST : 0); t < issued_v; ++t)
-          mbar_wait_drain(&bars->v_full[t % C::VST], (t / C::VST) & 1, lim);
-        if (!p.debug_stall) mbar_wait_drain(&bars->q_full, 0, lim);
-      }
-    }
-  } else if (SKIPV && warp == 10) {
-    // ======================================================== V producer (V skipping)
-    if (lane == 0 && n > 0) {
-      prefetch_tensormap(&tmV);
-      int vc = 0;   // V tiles loaded
-      bool ok = true;
-      for (int t = 0; ok && t < n; ++t) {
-        bool need = false;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          if (t < tb[e] || t >= te[e]) continue;
-          const int tl = t - tb[e];
-          if (!mbar_wait(&bars->dq_full[e][tl % C::DQ], (tl / C::DQ) & 1, abort, lim)) {
-            ok = false;
-            break;
-          }
-          need = need || *reinterpret_cast<volatile int*>(&bars->dval[e][tl % C::DQ]) != 0;
-          mbar_arrive(&bars->dq_empty[e][tl % C::DQ]);
+            tma_load_3d(k_smem + ks * C::T_BYTES + hf * C::T_HALF, &tmK, &bars->k_full[ks],
+                        hf * 64, j * BLK, b * p.Hkv + kvh);
+          ++issued_k;
+          if (SKIPV) continue;   // warp 10 loads V
+          const int vs = t % C::VST;
+          if (!mbar_wait(&bars->v_empty[vs], ((t / C::VST) & 1) ^ 1, abort, lim)) break;
+          mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
+          for (int hf = 0; hf < C::HALVES; ++hf)
+            tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
+                        hf * 64, j * BLK, b * p.Hkv + kvh);
+          ++issued_v;
         }
-        if (!ok || !need) continue;
-        const int vs = vc % C::VST;
-        if (!mbar_wait(&bars->v_empty[vs], ((vc / C::VST) & 1) ^ 1, abort, lim)) break;
-        mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
-        const int j = col_at(t);
-        for (int hf = 0; hf < C::HALVES; ++hf)
-          tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
-                      hf * 64, j * BLK, b * p.Hkv + kvh);
-        ++vc;
-      }
-      if (*abort)
-        for (int x = (vc > C::VST ? vc - C::VST : 0); x < vc; ++x)
-          mbar_wait_drain(&bars->v_full[x % C::VST], (x / C::VST) & 1, lim);
-    }
-  } else if (warp == 1) {
-    // ======================================================== MMA issuer
-    if (lane == 0 && n > 0) {
-      constexpr uint32_t IDESC1 = idesc_bf16_f32(128, BLK, 0, 0);
-      constexpr uint32_t IDESC2 = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_addr = smem_u32(q_smem);
-      const uint32_t k_addr = smem_u32(k_smem);
-      const uint32_t v_addr = smem_u32(v_smem);
-      bool ok = mbar_wait(&bars->q_full, 0, abort, lim);
-      tc_fence_after();
-      // S_e = Q_e K_t^T into TMEM columns [256 e, 256 e + 128)
-      auto bmm1 = [&](int e, int t) {
-        const int ks = t % C::KST;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a = q_addr + e * C::Q_BYTES + (kk / 4) * C::Q_HALF + (kk % 4) * 32;
-          const uint32_t bb = k_addr + ks * C::T_BYTES + (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(tmem + 256 * e, smem_desc(a, 16, 1024, 2), smem_desc(bb, 16, 1024, 2), IDESC1,
-                 kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars->s_full[e]);
-      };
-      // O_e += P_e V, P_e in TMEM over S_e, V in ring slot vs
-      auto bmm2 = [&](int e, int vs, int first) {
-#pragma unroll
-        for (int kk = 0; kk < BLK / 16; ++kk) {
-          const uint32_t bb = v_addr + vs * C::T_BYTES + kk * (16 * 128);
-          mma_ts(tmem + 256 * e + 128, tmem + 256 * e + kk * 8, smem_desc(bb, C::T_HALF, 1024, 2),
-                 IDESC2, (!first || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&bars->o_done[e]);
-      };
-      if (ok) {
-        ok = mbar_wait(&bars->k_full[0], 0, abort, lim);
-        tc_fence_after();
-        if (ok) {
-          if (tb[0] == 0 && te[0] > 0) bmm1(0, 0);
-          if (tb[1] == 0 && te[1] > 0) bmm1(1, 0);
-          mma_commit(&bars->k_empty[0]);
+        if (*abort) {
+          for (int t = (issued_k > C::KST ? issued_k - C::KST : 0); t < issued_k; ++t)
+            mbar_wait_drain(&bars->k_full[t % C::KST], (t / C::KST) & 1, lim);
+          for (int t = (issued_v > C::VST ? issued_v - C::VST : 0); t < issued_v; ++t)
+            mbar_wait_drain(&bars->v_full[t % C::VST], (t / C::VST) & 1, lim);
+          if (!p.debug_stall) mbar_wait_drain(&bars->q_full, 0, lim);
         }
       }
-      int kept[2] = {0, 0};
-      int vc = 0;   // V tiles loaded so far (V skipping: only the kept steps')
-      for (int t = 0; ok && t < n; ++t) {
-        const int vi = SKIPV ? vc : t;
-        const int vs = vi % C::VST;
-        bool v_ready = false;
-        bool k_next = false;        // K_{t+1} waited for
-        const bool more = t + 1 < n;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          if (t >= tb[e] && t < te[e]) {   // this slot takes part in step t
-            if (!mbar_wait(&bars->p_ready[e], (t - tb[e]) & 1, abort, lim)) { ok = false; break; }
-            tc_fence_after();
-            const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[e]);
-            if (!skip) {
-              if (!v_ready) {
-                if (!mbar_wait(&bars->v_full[vs], (vi / C::VST) & 1, abort, lim)) { ok = false; break; }
-                tc_fence_after();
-                v_ready = true;
-              }
-              bmm2(e, vs, kept[e] == 0);
-              ++kept[e];
+    } else if (SKIPV && warp == 2) {
+      // ======================================================== V producer (V skipping)
+      if (lane == 0 && n > 0) {
+        prefetch_tensormap(&tmV);
+        int vc = 0;   // V tiles loaded
+        bool ok = true;
+        for (int t = 0; ok && t < n; ++t) {
+          bool need = false;
+  #pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            if (t < tb[e] || t >= te[e]) continue;
+            const int tl = t - tb[e];
+            if (!mbar_wait(&bars->dq_full[e][tl % C::DQ], (tl / C::DQ) & 1, abort, lim)) {
+              ok = false;
+              break;
             }
+            need = need || *reinterpret_cast<volatile int*>(&bars->dval[e][tl % C::DQ]) != 0;
+            mbar_arrive(&bars->dq_empty[e][tl % C::DQ]);
           }
-          if (t + 1 >= tb[e] && t + 1 < te[e]) {
-            if (!k_next) {   // first use of K_{t+1}
-              const int ks = (t + 1) % C::KST;
-              if (!mbar_wait(&bars->k_full[ks], ((t + 1) / C::KST) & 1, abort, lim)) { ok = false; break; }
-              tc_fence_after();
-              k_next = true;
-            }
-            bmm1(e, t + 1);
-          }
-        }
-        if (!ok) break;
-        if (more) mma_commit(&bars->k_empty[(t + 1) % C::KST]);
-        // release V_t: consumed (or not needed) by both heads; with V skipping
-        // a step that no slot keeps has no V tile
-        if (v_ready) {
-          mma_commit(&bars->v_empty[vs]);
+          if (!ok || !need) continue;
+          const int vs = vc % C::VST;
+          if (!mbar_wait(&bars->v_empty[vs], ((vc / C::VST) & 1) ^ 1, abort, lim)) break;
+          mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
+          const int j = col_at(t);
+          for (int hf = 0; hf < C::HALVES; ++hf)
+            tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
+                        hf * 64, j * BLK, b * p.Hkv + kvh);
           ++vc;
-        } else if (!SKIPV) {
-          if (!mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) break;
-          mbar_arrive(&bars->v_empty[vs]);
         }
+        if (*abort)
+          for (int x = (vc > C::VST ? vc - C::VST : 0); x < vc; ++x)
+            mbar_wait_drain(&bars->v_full[x % C::VST], (x / C::VST) & 1, lim);
       }
-      mma_commit(&bars->drain);
-      mbar_wait_drain(&bars->drain, 0, lim);
+    } else if (warp == 1) {
+      // ======================================================== MMA issuer
+      if (lane == 0 && n > 0) {
+        constexpr uint32_t IDESC1 = idesc_bf16_f32(128, BLK, 0, 0);
+        constexpr uint32_t IDESC2 = idesc_bf16_f32(128, D, 0, 1);
+        const uint32_t q_addr = smem_u32(q_smem);
+        const uint32_t k_addr = smem_u32(k_smem);
+        const uint32_t v_addr = smem_u32(v_smem);
+        bool ok = mbar_wait(&bars->q_full, 0, abort, lim);
+        tc_fence_after();
+        // S_e = Q_e K_t^T into TMEM columns [256 e, 256 e + 128)
+        auto bmm1 = [&](int e, int t) {
+          const int ks = t % C::KST;
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t a = q_addr + e * C::Q_BYTES + (kk / 4) * C::Q_HALF + (kk % 4) * 32;
+            const uint32_t bb = k_addr + ks * C::T_BYTES + (kk / 4) * C::T_HALF + (kk % 4) * 32;
+            mma_ss(tmem + 256 * e, smem_desc(a, 16, 1024, 2), smem_desc(bb, 16, 1024, 2), IDESC1,
+                   kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars->s_full[e]);
+        };
+        // O_e += P_e V, P_e in TMEM over S_e, V in ring slot vs
+        auto bmm2 = [&](int e, int vs, int first) {
+  #pragma unroll
+          for (int kk = 0; kk < BLK / 16; ++kk) {
+            const uint32_t bb = v_addr + vs * C::T_BYTES + kk * (16 * 128);
+            mma_ts(tmem + 256 * e + 128, tmem + 256 * e + kk * 8, smem_desc(bb, C::T_HALF, 1024, 2),
+                   IDESC2, (!first || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bars->o_done[e]);
+        };
+        if (ok) {
+          ok = mbar_wait(&bars->k_full[0], 0, abort, lim);
+          tc_fence_after();
+          if (ok) {
+            if (tb[0] == 0 && te[0] > 0) bmm1(0, 0);
+            if (tb[1] == 0 && te[1] > 0) bmm1(1, 0);
+            mma_commit(&bars->k_empty[0]);
+          }
+        }
+        int kept[2] = {0, 0};
+        int vc = 0;   // V tiles loaded so far (V skipping: only the kept steps')
+        for (int t = 0; ok && t < n; ++t) {
+          const int vi = SKIPV ? vc : t;
+          const int vs = vi % C::VST;
+          bool v_ready = false;
+          bool k_next = false;        // K_{t+1} waited for
+          const bool more = t + 1 < n;
+  #pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            if (t >= tb[e] && t < te[e]) {   // this slot takes part in step t
+              if (!mbar_wait(&bars->p_ready[e], (t - tb[e]) & 1, abort, lim)) { ok = false; break; }
+              tc_fence_after();
+              const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[e]);
+              if (!skip) {
+                if (!v_ready) {
+                  if (!mbar_wait(&bars->v_full[vs], (vi / C::VST) & 1, abort, lim)) { ok = false; break; }
+                  tc_fence_after();
+                  v_ready = true;
+                }
+                bmm2(e, vs, kept[e] == 0);
+                ++kept[e];
+              }
+            }
+            if (t + 1 >= tb[e] && t + 1 < te[e]) {
+              if (!k_next) {   // first use of K_{t+1}
+                const int ks = (t + 1) % C::KST;
+                if (!mbar_wait(&bars->k_full[ks], ((t + 1) / C::KST) & 1, abort, lim)) { ok = false; break; }
+                tc_fence_after();
+                k_next = true;
+              }
+              bmm1(e, t + 1);
+            }
+          }
+          if (!ok) break;
+          if (more) mma_commit(&bars->k_empty[(t + 1) % C::KST]);
+          // release V_t: consumed (or not needed) by both heads; with V skipping
+          // a step that no slot keeps has no V tile
+          if (v_ready) {
+            mma_commit(&bars->v_empty[vs]);
+            ++vc;
+          } else if (!SKIPV) {
+            if (!mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) break;
+            mbar_arrive(&bars->v_empty[vs]);
+          }
+        }
+        mma_commit(&bars->drain);
+        mbar_wait_drain(&bars->drain, 0, lim);
+      }
     }
   } else {
-    // ======================================================== softmax warps
-    const int e = (warp - 2) / 4;           // which slot of the pair
-    const int sw = (warp - 2) % 4;
-    const int quarter = warp % 4;
-    const int row = quarter * 32 + lane;
-    // this slot's values as scalars (a runtime index would put the arrays in
-    // local memory)
-    const int i = e ? is[1] : is[0];
-    const int r0 = i * BLK;
-    const int h = e ? hs[1] : hs[0];
-    const int t_first = e ? tb[1] : tb[0];
-    const int ne = (e ? te[1] : te[0]) - t_first;
-    // key tile of this slot's t-th visit: u0 + du * t into the CSR row (or
-    // the tile index itself without one)
-    const int du = p.reverse ? -1 : 1;
-    const int u0 = p.reverse ? n - 1 - t_first : t_first;
-    const bool valid = r0 + row < lenb;    // votes, and gets an output
-    const bool in_buf = r0 + row < p.N;    // written (padding rows as zeros)
-    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t s_col = 256 * e, o_col = 256 * e + 128;
-    float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
-    int kept = 0;
-    bool ok = true;
-    for (int t = 0; t < ne; ++t) {       // t counts this slot's tiles
-      const int u = u0 + du * t;
-      const int j = cols ? cols[u] : u;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[e], t & 1, abort, lim))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t r[BLK];
-#pragma unroll
-      for (int c0 = 0; c0 < BLK; c0 += 32)
-        tmem_ld32(lane_addr + s_col + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
-      tmem_wait_ld();
-      const int k0 = j * BLK;
-      if (k0 + BLK > lenb || (p.causal && j == i)) {
-        const int qpos = r0 + row;
-#pragma unroll
-        for (int c = 0; c < BLK; ++c) {
-          const int key = k0 + c;
-          if (key >= lenb || (p.causal && key > qpos)) r[c] = __float_as_uint(-INFINITY);
-        }
-      }
-      const float mx = row_max<BLK>(reinterpret_cast<const float*>(r));
-      const float mt = mx * p.scale_log2;
-      int skip = 0;
-      if (p.use_skip) {
-        const bool pass = !valid || (mt - m_run < p.thr_log2);
-        const bool wpass = __all_sync(0xffffffffu, pass);
-        if (lane == 0) {
-          bars->vote[e][t & 1][sw] = wpass ? 1 : 0;
-          mbar_arrive(&bars->vote_bar[e][t & 1]);
-        }
-        __syncwarp();
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(&bars->vote_bar[e][t & 1], (t >> 1) & 1, abort, lim))) {
+    setmaxnreg_inc<C::REG_HIGH>();
+    {
+      // ======================================================== softmax warps
+      const int e = (warp - 4) / 4;           // which slot of the pair
+      const int sw = (warp - 4) % 4;
+      const int quarter = warp % 4;
+      const int row = quarter * 32 + lane;
+      // this slot's values as scalars (a runtime index would put the arrays in
+      // local memory)
+      const int i = e ? is[1] : is[0];
+      const int r0 = i * BLK;
+      const int h = e ? hs[1] : hs[0];
+      const int t_first = e ? tb[1] : tb[0];
+      const int ne = (e ? te[1] : te[0]) - t_first;
+      // key tile of this slot's t-th visit: u0 + du * t into the CSR row (or
+      // the tile index itself without one)
+      const int du = p.reverse ? -1 : 1;
+      const int u0 = p.reverse ? n - 1 - t_first : t_first;
+      const bool valid = r0 + row < lenb;    // votes, and gets an output
+      const bool in_buf = r0 + row < p.N;    // written (padding rows as zeros)
+      const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t s_col = 256 * e, o_col = 256 * e + 128;
+      float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
+      int kept = 0;
+      bool ok = true;
+      for (int t = 0; t < ne; ++t) {       // t counts this slot's tiles
+        const int u = u0 + du * t;
+        const int j = cols ? cols[u] : u;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[e], t & 1, abort, lim))) {
           ok = false;
           break;
         }
-        volatile int* vv = bars->vote[e][t & 1];
-        skip = vv[0] & vv[1] & vv[2] & vv[3];
-      }
-      if (SKIPV) {   // the decision to the V producer, before any exponential
-        if (sw == 0 && lane == 0) {
-          const int dq = t % C::DQ;
-          if (mbar_wait(&bars->dq_empty[e][dq], ((t / C::DQ) & 1) ^ 1, abort, lim)) {
-            bars->dval[e][dq] = skip ? 0 : 1;
-            mbar_arrive(&bars->dq_full[e][dq]);
+        tc_fence_after();
+        uint32_t r[BLK];
+  #pragma unroll
+        for (int c0 = 0; c0 < BLK; c0 += 32)
+          tmem_ld32(lane_addr + s_col + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
+        tmem_wait_ld();
+        const int k0 = j * BLK;
+        if (k0 + BLK > lenb || (p.causal && j == i)) {
+          const int qpos = r0 + row;
+  #pragma unroll
+          for (int c = 0; c < BLK; ++c) {
+            const int key = k0 + c;
+            if (key >= lenb || (p.causal && key > qpos)) r[c] = __float_as_uint(-INFINITY);
           }
         }
-        if (__any_sync(0xffffffffu, *abort != 0)) {
-          ok = false;
-          break;
-        }
-      }
-      m_run = fmaxf(m_run, mt);
-      if (sw == 0 && lane == 0 && p.tile_status && (unsigned)j < (unsigned)p.nk)
-        p.tile_status[(((int64_t)b * p.Hq + h) * p.nq + i) * p.nk + j] = skip ? 1 : 2;
-      if (!skip) {
-        if (kept > 0) {
-          // S_e holds this tile, so BMM2 of the previous kept tile has finished
-          // reading P; wait for it to land in O before O may be rescaled
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[e], (kept - 1) & 1, abort, lim))) {
+        const float mx = row_max<BLK>(reinterpret_cast<const float*>(r));
+        const float mt = mx * p.scale_log2;
+        int skip = 0;
+        if (p.use_skip) {
+          const bool pass = !valid || (mt - m_run < p.thr_log2);
+          const bool wpass = __all_sync(0xffffffffu, pass);
+          if (lane == 0) {
+            bars->vote[e][t & 1][sw] = wpass ? 1 : 0;
+            mbar_arrive(&bars->vote_bar[e][t & 1]);
+          }
+          __syncwarp();
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait(&bars->vote_bar[e][t & 1], (t >> 1) & 1, abort, lim))) {
             ok = false;
             break;
           }
-          tc_fence_after();
+          volatile int* vv = bars->vote[e][t & 1];
+          skip = vv[0] & vv[1] & vv[2] & vv[3];
         }
-        float alpha = 1.f;
-        bool rescale = false;
-        if (kept == 0) {
-          m_ref = m_run;
-        } else if (m_run > m_ref + C::TAU) {
-          alpha = fast_exp2(m_ref - m_run);
-          rescale = true;
-          m_ref = m_run;
-        }
-        const float shift = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c0 = 0; c0 < BLK; c0 += 32) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(r[c0 + c]), p.scale_log2, -shift));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(r[c0 + c + 1]), p.scale_log2, -shift));
-            rs8[(c / 2) & 7] += p0 + p1;
-            pk[c / 2] = pack_bf16x2(p0, p1);
+        if (SKIPV) {   // the decision to the V producer, before any exponential
+          if (sw == 0 && lane == 0) {
+            const int dq = t % C::DQ;
+            if (mbar_wait(&bars->dq_empty[e][dq], ((t / C::DQ) & 1) ^ 1, abort, lim)) {
+              bars->dval[e][dq] = skip ? 0 : 1;
+              mbar_arrive(&bars->dq_full[e][dq]);
+            }
           }
-          tmem_st16(lane_addr + s_col + c0 / 2, pk);
+          if (__any_sync(0xffffffffu, *abort != 0)) {
+            ok = false;
+            break;
+          }
         }
-        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) +
-                         ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-        l = l * alpha + rs;
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t ro[32];
+        m_run = fmaxf(m_run, mt);
+        if (sw == 0 && lane == 0 && p.tile_status && (unsigned)j < (unsigned)p.nk)
+          p.tile_status[(((int64_t)b * p.Hq + h) * p.nq + i) * p.nk + j] = skip ? 1 : 2;
+        if (!skip) {
+          if (kept > 0) {
+            // S_e holds this tile, so BMM2 of the previous kept tile has finished
+            // reading P; wait for it to land in O before O may be rescaled
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[e], (kept - 1) & 1, abort, lim))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          float alpha = 1.f;
+          bool rescale = false;
+          if (kept == 0) {
+            m_ref = m_run;
+          } else if (m_run > m_ref + C::TAU) {
+            alpha = fast_exp2(m_ref - m_run);
+            rescale = true;
+            m_ref = m_run;
+          }
+          const float shift = (m_ref == -INFINITY) ? 0.f : m_ref;
+          // P = exp2(S * scale_log2 - shift), two columns per packed FMA and
+          // row-sum add, written back over S as bf16 pairs
+          const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+          const float2 sh2 = make_float2(-shift, -shift);
+          float2 rs4[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+  #pragma unroll
+          for (int c0 = 0; c0 < BLK; c0 += 32) {
+            uint32_t pk[16];
+  #pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const float2 x = ffma2(make_float2(__uint_as_float(r[c0 + c]),
+                                                 __uint_as_float(r[c0 + c + 1])), sc2, sh2);
+              const float2 pv = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+              rs4[(c / 2) & 3] = fadd2(rs4[(c / 2) & 3], pv);
+              pk[c / 2] = pack_bf16x2(pv.x, pv.y);
+            }
+            tmem_st16(lane_addr + s_col + c0 / 2, pk);
+          }
+          const float2 rs2 = fadd2(fadd2(rs4[0], rs4[1]), fadd2(rs4[2], rs4[3]));
+          const float rs = rs2.x + rs2.y;
+          l = l * alpha + rs;
+          if (__any_sync(0xffffffffu, rescale)) {
+  #pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t ro[32];
+              tmem_ld32(lane_addr + o_col + c0, ro);
+              tmem_wait_ld();
+  #pragma unroll
+              for (int c = 0; c < 32; ++c) ro[c] = __float_as_uint(__uint_as_float(ro[c]) * alpha);
+              tmem_st32(lane_addr + o_col + c0, ro);
+            }
+          }
+          tmem_wait_st();
+          ++kept;
+        }
+        if (sw == 0 && lane == 0) bars->skip_flag[e] = skip;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_ready[e]);
+      }
+      // ---- epilogue
+      if (ok && kept > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[e], (kept - 1) & 1, abort, lim)))
+          ok = false;
+        tc_fence_after();
+      }
+      if (ok) {
+        const int64_t orow = ((int64_t)b * p.Hq + h) * p.N + r0 + row;
+        __nv_bfloat16* dst = p.o + orow * D;
+        const bool have = valid && kept > 0 && l > 0.f;
+        const float inv_l = have ? 1.f / l : 0.f;
+  #pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t ro[32];
+          if (kept > 0) {
             tmem_ld32(lane_addr + o_col + c0, ro);
             tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) ro[c] = __float_as_uint(__uint_as_float(ro[c]) * alpha);
-            tmem_st32(lane_addr + o_col + c0, ro);
+          }
+          if (in_buf) {
+            uint32_t w[16];
+  #pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const float a0 = have ? __uint_as_float(ro[c]) * inv_l : 0.f;
+              const float a1 = have ? __uint_as_float(ro[c + 1]) * inv_l : 0.f;
+              w[c / 2] = pack_bf16x2(a0, a1);
+            }
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+  #pragma unroll
+            for (int v = 0; v < 4; ++v)
+              d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
           }
         }
-        tmem_wait_st();
-        ++kept;
+        if (in_buf && p.lse)
+          p.lse[orow] = have ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       }
-      if (sw == 0 && lane == 0) bars->skip_flag[e] = skip;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_ready[e]);
     }
-    // ---- epilogue
-    if (ok && kept > 0) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[e], (kept - 1) & 1, abort, lim)))
-        ok = false;
-      tc_fence_after();
-    }
-    if (ok) {
-      const int64_t orow = ((int64_t)b * p.Hq + h) * p.N + r0 + row;
-      __nv_bfloat16* dst = p.o + orow * D;
-      const bool have = valid && kept > 0 && l > 0.f;
-      const float inv_l = have ? 1.f / l : 0.f;
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t ro[32];
-        if (kept > 0) {
-          tmem_ld32(lane_addr + o_col + c0, ro);
-          tmem_wait_ld();
-        }
-        if (in_buf) {
-          uint32_t w[16];
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float a0 = have ? __uint_as_float(ro[c]) * inv_l : 0.f;
-            const float a1 = have ? __uint_as_float(ro[c + 1]) * inv_l : 0.f;
-            w[c / 2] = pack_bf16x2(a0, a1);
-          }
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-        }
-      }
-      if (in_buf && p.lse)
-        p.lse[orow] = have ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-    }
+
   }
 
   tc_fence_before();
@@ -578,7 +597,15 @@ static cudaError_t launch_pair(const CUtensorMap& tq, const CUtensorMap& tk,
   cudaError_t e = cudaFuncSetAttribute(prefill_pair_kernel<D, SKIPV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  prefill_pair_kernel<D, SKIPV><<<grid, SKIPV ? 352 : 320, C::SMEM, stream>>>(tq, tk, tv, p);
+  static_assert(128 * C::REG_LOW + 256 * C::REG_HIGH == C::THREADS * C::REG_LAUNCH,
+                "register split must equal the launch allocation");
+  // setmaxnreg.inc waits until the block's pool has the registers; launch only
+  // when the compiled kernel reserves the REG_LAUNCH the split is built on
+  cudaFuncAttributes attr;
+  e = cudaFuncGetAttributes(&attr, prefill_pair_kernel<D, SKIPV>);
+  if (e != cudaSuccess) return e;
+  if (attr.numRegs != C::REG_LAUNCH) return cudaErrorInvalidConfiguration;
+  prefill_pair_kernel<D, SKIPV><<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 

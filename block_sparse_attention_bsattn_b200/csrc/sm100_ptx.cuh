@@ -244,6 +244,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Per-warpgroup register reallocation (every thread of the warpgroup executes
+// the same one).  dec returns registers to the block's pool; inc waits until
+// the pool holds them, so the split must not exceed what the block was
+// launched with.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
 // max of three floats in one instruction (sm_100's three-input max.f32)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
@@ -265,6 +278,28 @@ __device__ __forceinline__ float row_max(const float* v) {
     for (int x = 0; x < 8; ++x) m[x] = fmax3(m[x], v[c + x], c + 8 < N ? v[c + 8 + x] : -INFINITY);
   const float a = fmax3(m[0], m[1], m[2]), b = fmax3(m[3], m[4], m[5]);
   return fmax3(a, b, fmaxf(m[6], m[7]));
+}
+
+// Two-lane fp32 arithmetic (sm_100's packed f32x2 FMA and add): one
+// instruction for two independent lanes.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
