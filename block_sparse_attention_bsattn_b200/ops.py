@@ -45,6 +45,9 @@ _lib.bsattn_fwd_prefill.restype = _I
 _lib.bsattn_fwd_prefill_ex.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F,
                                        _P, _P, _P, _I, _P, _P, ctypes.c_uint, _P, _P]
 _lib.bsattn_fwd_prefill_ex.restype = _I
+_lib.bsattn_fwd_prefill_host.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                         _F, _I, _F, _P, _P, _P, _I, _I, _P, _P]
+_lib.bsattn_fwd_prefill_host.restype = _I
 _lib.bsattn_decode_workspace_size.argtypes = [_I, _I, _I, _I]
 _lib.bsattn_decode_workspace_size.restype = _SZ
 _lib.bsattn_fwd_decode.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _F, _I,
@@ -64,7 +67,8 @@ DECODE_SINK_SEED = 0x1
 
 EXPORTED = ("bsattn_status_string", "bsattn_version", "bsattn_debug_set", "bsattn_debug_trace",
             "bsattn_build_index",
-            "bsattn_fwd_prefill", "bsattn_fwd_prefill_ex", "bsattn_decode_workspace_size",
+            "bsattn_fwd_prefill", "bsattn_fwd_prefill_ex", "bsattn_fwd_prefill_host",
+            "bsattn_decode_workspace_size",
             "bsattn_fwd_decode", "bsattn_fwd_decode_ex",
             "bsattn_fwd_decode_noalloc")
 
@@ -189,6 +193,40 @@ def bsattn_fwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
     if rc:
         raise BsattnError(rc, "bsattn_fwd_prefill")
     return o, lse
+
+
+def bsattn_fwd_prefill_host(hq: torch.Tensor, hk: torch.Tensor, hv: torch.Tensor,
+                            ho: torch.Tensor, dq: torch.Tensor, dk: torch.Tensor,
+                            dv: torch.Tensor, do: torch.Tensor, block: int,
+                            scale: Optional[float] = None, causal: bool = False,
+                            lam: float = 0.0, row_ptr: Optional[torch.Tensor] = None,
+                            col_idx: Optional[torch.Tensor] = None, mask_heads: int = 1,
+                            row_order: Optional[torch.Tensor] = None,
+                            kv_heads_per_chunk: int = 1, status: Optional[torch.Tensor] = None,
+                            stream=None) -> None:
+    """Prefill of host (pinned) hq/hk/hv into host ho, staged through the
+    device tensors dq/dk/dv/do with copies and kernels overlapped per chunk of
+    KV heads.  Only enqueues: synchronise the stream before reading ho."""
+    for t, name in ((hq, "hq"), (hk, "hk"), (hv, "hv"), (ho, "ho")):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name}: expected a contiguous host bf16 tensor with 4 dims")
+    for t, name in ((dq, "dq"), (dk, "dk"), (dv, "dv"), (do, "do")):
+        _check(t, name, torch.bfloat16, 4)
+    B, Hq, N, d = hq.shape
+    Hkv = hk.shape[1]
+    if dq.shape != hq.shape or do.shape != hq.shape or ho.shape != hq.shape or \
+            dk.shape != hk.shape or dv.shape != hk.shape or hv.shape != hk.shape:
+        raise ValueError("staging and host shapes must match")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = _lib.bsattn_fwd_prefill_host(
+        ctypes.c_void_p(hq.data_ptr()), ctypes.c_void_p(hk.data_ptr()),
+        ctypes.c_void_p(hv.data_ptr()), ctypes.c_void_p(ho.data_ptr()), _ptr(dq), _ptr(dk),
+        _ptr(dv), _ptr(do), B, Hq, Hkv, N, d, int(block), float(scale), int(causal), float(lam),
+        _ptr(row_ptr), _ptr(col_idx), _ptr(row_order), int(mask_heads), int(kv_heads_per_chunk),
+        _ptr(status), _stream(stream))
+    if rc:
+        raise BsattnError(rc, "bsattn_fwd_prefill_host")
 
 
 def bsattn_decode_workspace_size(B: int, Hq: int, d: int, num_splits: int) -> int:

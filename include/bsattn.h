@@ -186,6 +186,41 @@ int bsattn_fwd_prefill_ex(const void *q, const void *k, const void *v, void *o, 
                           int32_t *d_status, cudaStream_t stream);
 
 /*
+ * bsattn_fwd_prefill_host -- bsattn_fwd_prefill for inputs in host memory,
+ * with the transfers overlapped with the kernels.  The pages have no
+ * counterpart of this entry point: it serves callers that keep Q, K and V on
+ * the host, for whom the copies in and out take longer than the attention.
+ *
+ * The batch is cut into chunks of one sequence and kv_heads_per_chunk KV
+ * heads (with their query heads); each chunk is copied host -> device on an
+ * internal stream, computed by bsattn_fwd_prefill on `stream` once its copies
+ * have landed, and its O copied device -> host on a second internal stream,
+ * so copies in, kernels and copies out of different chunks run at once.  The
+ * call only enqueues work: `stream` completes after the last copy out.
+ *
+ *   h_q, h_k, h_v   host inputs, layouts as in bsattn_fwd_prefill; page-locked
+ *                   (cudaHostAlloc / pinned) for the copies to overlap
+ *   h_o             host output [B][Hq][N][d] bf16
+ *   d_q, d_k, d_v, d_o  device staging of the full tensors' sizes, owned by
+ *                   the caller; their contents are overwritten
+ *   row_ptr, col_idx, row_order, mask_heads   as in bsattn_fwd_prefill (device
+ *                   memory; per-head masks are sliced per chunk)
+ *   kv_heads_per_chunk  divides Hkv; 1 gives the finest overlap
+ *
+ * The caller must not touch the host or staging buffers before `stream`
+ * completes.  The first call on a device creates two streams and a ring of
+ * events for it, kept until the process exits.  No LSE or tile status is
+ * produced.  Errors as in bsattn_fwd_prefill, plus BSATTN_ERR_INVALID_ARG for
+ * a chunk size that does not divide Hkv.
+ */
+int bsattn_fwd_prefill_host(const void *h_q, const void *h_k, const void *h_v, void *h_o,
+                            void *d_q, void *d_k, void *d_v, void *d_o, int B, int Hq, int Hkv,
+                            int N, int d, int block, float scale, int causal, float lambda,
+                            const int32_t *row_ptr, const int32_t *col_idx,
+                            const int32_t *row_order, int mask_heads, int kv_heads_per_chunk,
+                            int32_t *d_status, cudaStream_t stream);
+
+/*
  * bsattn_decode_workspace_size -- bytes of scratch bsattn_fwd_decode needs:
  * per (batch, query head, split) d fp32 partial outputs plus the split's
  * running max and row sum.

@@ -117,6 +117,20 @@ def test_option_bits_validation(lib):
     assert dec(0x2) == -1 and dec(0x1, q=0) == -1
 
 
+def test_host_pipeline_validation(lib):
+    """bsattn_fwd_prefill_host rejects bad arguments before touching a device."""
+    f = lib.bsattn_fwd_prefill_host
+
+    def call(chunk=1, d=128, hq=0x1000):
+        return f(P(hq) if hq else None, P(0x2000), P(0x3000), P(0x4000), P(0x5000), P(0x6000),
+                 P(0x7000), P(0x8000), 1, 8, 2, 256, d, 128, ctypes.c_float(0.1), 1,
+                 ctypes.c_float(0.0), None, None, None, 1, chunk, None, None)
+    assert call(hq=0) == -1
+    assert call(chunk=0) == -1
+    assert call(chunk=3) == -1          # does not divide the two KV heads
+    assert call(d=96) == -2
+
+
 def test_index_host_validation(lib):
     f = lib.bsattn_build_index
     assert f(None, 1, 4, 4, 64, 64, 0, P(0x1000), P(0x2000), 16, P(0x3000), None, None, None) == -1

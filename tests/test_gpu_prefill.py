@@ -255,6 +255,41 @@ def test_varlen_key_padding(hq, hkv, block, causal, masked, reverse):
         assert torch.isneginf(lse[b, :, L:]).all()
 
 
+@pytest.mark.parametrize("masked", [None, "shared", "per_head"])
+@pytest.mark.parametrize("chunk", [1, 2])
+def test_host_pipeline_equals_device_path(masked, chunk):
+    """bsattn_fwd_prefill_host (host buffers, per-chunk copies overlapped with
+    the kernels) gives exactly the output of the device path."""
+    ops = _ops()
+    B, Hq, Hkv, N, block = 2, 8, 2, 5 * 128 + 37, 128
+    q, k, v = inputs.blasst_prefill_qkv(B, Hq, Hkv, N, 128, "cpu", 44)
+    lam = 0.02
+    rp = ci = order = None
+    mh = 1
+    if masked:
+        nb = -(-N // block)
+        heads = 1 if masked == "shared" else Hq
+        rng = np.random.default_rng(6)
+        m = (rng.random((heads, nb, nb)) < 0.6).astype(np.uint8)
+        m[:, np.arange(nb), np.arange(nb)] = 1
+        rp, ci, _, order = ops.bsattn_build_index(torch.as_tensor(m).cuda(), block, block, True,
+                                                  with_order=True)
+        mh = heads
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    ref, _ = ops.bsattn_fwd_prefill(qd, kd, vd, block, None, True, lam, rp, ci, mh,
+                                    row_order=order, want_lse=False)
+    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    ho = torch.empty_like(q).pin_memory()
+    sq, sk, sv, so = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd), \
+        torch.empty_like(qd)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ops.bsattn_fwd_prefill_host(hq, hk, hv, ho, sq, sk, sv, so, block, None, True, lam, rp, ci,
+                                mh, row_order=order, kv_heads_per_chunk=chunk, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(ho, ref.cpu())
+
+
 def test_short_sequence_single_partial_tile():
     q, k, v = inputs.normal_qkv(1, 2, 2, 50, 128, "cpu", 3)
     w = inputs.Workload("short", 1, 2, 2, 50, 128, 128, True, "prefill", 1 / math.sqrt(128), None,
