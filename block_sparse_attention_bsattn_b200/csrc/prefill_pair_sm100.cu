@@ -120,8 +120,14 @@ __global__ void __launch_bounds__(384, 1)
     const int PH = p.Hq / 2;
     int i, bp;
     if (p.row_order) {
-      bp = (int)(blockIdx.x / p.nq);
-      i = p.row_order[(int)(blockIdx.x % p.nq)];
+      // KV-head-major like the causal order below, the builder's row order
+      // (longest rows first) inside a KV head, its head pairs interleaved
+      const int PPK = (p.Hq / p.Hkv) / 2;
+      const int per_kv = p.nq * PPK;
+      const int gi = (int)(blockIdx.x / (unsigned)per_kv);
+      const int rem = (int)(blockIdx.x - (unsigned)gi * per_kv);
+      i = p.row_order[rem / PPK];
+      bp = gi * PPK + rem % PPK;
     } else if (p.causal) {
       // groups of KVG (batch, KV head) streams, one after another; inside a
       // group, longest query tile first across the group's head pairs
