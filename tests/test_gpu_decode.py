@@ -127,6 +127,14 @@ def test_varlen_cache_lengths(d, block, g, sink_seed):
     assert (o_c[4] == 0).all() and np.isneginf(lse_c[4]).all()   # an empty cache
 
 
+def test_long_cache():
+    """A 1,048,699-token cache (8,193 tiles, 16 splits of 513) for one
+    sequence and a GQA group of 4, against the oracle."""
+    q, k, v = inputs.blasst_decode_qkv(1, 4, 1, (1 << 20) + 123, 128, "cuda", 77)
+    _check(q, k, v, 128, 16, 1 / math.sqrt(128), inputs.lambda_for(10.0, (1 << 20) + 123),
+           what="1M-token cache")
+
+
 def test_more_splits_than_tiles():
     q, k, v = inputs.blasst_decode_qkv(1, 4, 1, 300, 128, "cpu", 9)
     _check(q, k, v, 128, 8, 1 / math.sqrt(128), 1e-2, what="empty splits")

@@ -290,6 +290,26 @@ def test_host_pipeline_equals_device_path(masked, chunk):
     assert torch.equal(ho, ref.cpu())
 
 
+def test_long_sequence_sampled():
+    """A 131,149-token causal prefill (1,025 query tiles, 1,050,625 tile-status
+    entries per head) with the skip on: sampled query tiles, including the
+    last and ragged one, against the oracle."""
+    B, Hq, Hkv, N = 1, 2, 1, 131072 + 77
+    q, k, v = inputs.blasst_prefill_qkv(B, Hq, Hkv, N, 128, "cuda", 321)
+    w = inputs.Workload("long", B, Hq, Hkv, N, 128, 128, True, "prefill", 1 / math.sqrt(128),
+                        None, q=q, k=k, v=v)
+    lam = inputs.lambda_for(10.0, N)
+    o, lse, st = _run_gpu(w, lam, None)
+    items = [(0, 0, 0), (0, 1, 513), (0, 0, 1024), (0, 1, 1024), (0, 0, 700)]
+    ref = oracle.prefill(q.cpu(), k.cpu(), v.cpu(), 128, w.scale, True, lam, items=items)
+    o_c, lse_c, st_c = o.float().cpu().numpy(), lse.cpu().numpy(), st.cpu().numpy()
+    for (b, h, i) in items:
+        rows = slice(i * 128, min(N, (i + 1) * 128))
+        compare_outputs(o_c[b, h, rows], ref["o"][b, h, rows], lse_c[b, h, rows],
+                        ref["lse"][b, h, rows], f"long item {(b, h, i)}")
+        compare_status(st_c[b, h, i], ref["status"][b, h, i], ref["margin"][b, h, i])
+
+
 def test_short_sequence_single_partial_tile():
     q, k, v = inputs.normal_qkv(1, 2, 2, 50, 128, "cpu", 3)
     w = inputs.Workload("short", 1, 2, 2, 50, 128, 128, True, "prefill", 1 / math.sqrt(128), None,
