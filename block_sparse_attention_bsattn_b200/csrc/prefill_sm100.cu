@@ -440,21 +440,24 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
         }
         const float shift = (m_ref == -INFINITY) ? 0.f : m_ref;
         if (in_tile) {
-          float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          // two columns per packed FMA and row-sum add
+          const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+          const float2 sh2 = make_float2(-shift, -shift);
+          float2 rs4[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
           for (int c0 = 0; c0 < CW; c0 += 32) {
             uint32_t pk[16];
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
-              const float p0 = fast_exp2(fmaf(s[c0 + c], p.scale_log2, -shift));
-              const float p1 = fast_exp2(fmaf(s[c0 + c + 1], p.scale_log2, -shift));
-              rs8[(c / 2) & 7] += p0 + p1;
-              pk[c / 2] = pack_bf16x2(p0, p1);
+              const float2 x = ffma2(make_float2(s[c0 + c], s[c0 + c + 1]), sc2, sh2);
+              const float2 pv = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+              rs4[(c / 2) & 3] = fadd2(rs4[(c / 2) & 3], pv);
+              pk[c / 2] = pack_bf16x2(pv.x, pv.y);
             }
             tmem_st16(lane_addr + C::S_COL + sb * 128 + (half * CW + c0) / 2, pk);
           }
-          const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) +
-                           ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+          const float2 rs2 = fadd2(fadd2(rs4[0], rs4[1]), fadd2(rs4[2], rs4[3]));
+          const float rs = rs2.x + rs2.y;
           l = l * alpha + rs;
           // rare: bring this half of the accumulated O to the new shift
           if (__any_sync(0xffffffffu, rescale)) {
