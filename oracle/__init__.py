@@ -19,6 +19,9 @@ Functions and the passages they follow:
   by the exact softmax over the executed tiles.
 * :func:`decode`       -- the same per split of the KV sequence, query tile =
   the GQA group of one token.
+* :func:`prefill_bwd`  -- the backward pass of sparsity-aware training (BLASST
+  page, section 3.3): the gradient of the forward's output with its executed
+  tiles held fixed; skipped tiles receive no gradient.
 """
 from __future__ import annotations
 
@@ -61,6 +64,9 @@ def bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_decode.argtypes = [P, P, P, i32, i32, i64, i32, i32, f64, f64, i32,
                                   P, P, P, P, i32, P]
     lib.oracle_decode.restype = i32
+    lib.oracle_prefill_bwd.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f64, i32,
+                                       P, P, P, P, P]
+    lib.oracle_prefill_bwd.restype = i32
     lib.oracle_num_threads.restype = i32
     return lib
 
@@ -182,6 +188,45 @@ def decode(q, k, v, block: int, scale: float, lam: float, num_splits: int,
     if rc != 0:
         raise OracleError(f"oracle_decode rc={rc}")
     return {"o": o, "lse": lse, "status": status, "margin": margin}
+
+
+def _f64(x) -> np.ndarray:
+    """bf16 tensor or bits (exact upcast), or any float tensor/array -> contiguous f64."""
+    if isinstance(x, np.ndarray) and x.dtype == np.uint16:
+        return np.ascontiguousarray(bf16_to_f64(x))
+    if not isinstance(x, np.ndarray):
+        import torch
+        if x.dtype == torch.bfloat16:
+            return np.ascontiguousarray(bf16_to_f64(x))
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def prefill_bwd(q, k, v, dout, block: int, scale: float, causal: bool, status,
+                seq_lens=None):
+    """Backward of :func:`prefill` for sparsity-aware training.  q, dout
+    [B,Hq,N,d], k/v [B,Hkv,N,d] (bf16 torch / uint16 bits, upcast exactly, or
+    any float array); status uint8 [B,Hq,nq,nk] as the forward returned it
+    (only tiles marked 2, executed, take part); seq_lens None or [B].  Returns
+    dict(dq [B,Hq,N,d], dk, dv [B,Hkv,N,d]) in f64."""
+    qd, kd, vd, dod = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Hq, N, d = qd.shape
+    Hkv = kd.shape[1]
+    nq = -(-N // block)
+    st = np.ascontiguousarray(np.asarray(status, dtype=np.uint8))
+    assert st.shape == (B, Hq, nq, nq) and dod.shape == qd.shape and vd.shape == kd.shape
+    sl = None
+    if seq_lens is not None:
+        sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32).reshape(B))
+    dq = np.zeros_like(qd)
+    dk = np.zeros_like(kd)
+    dv = np.zeros_like(vd)
+    rc = _load().oracle_prefill_bwd(_ptr(qd), _ptr(kd), _ptr(vd), _ptr(dod), B, Hq, Hkv, N, d,
+                                    block, float(scale), int(causal), _ptr(st), _ptr(sl),
+                                    _ptr(dq), _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise OracleError(f"oracle_prefill_bwd rc={rc}")
+    return {"dq": dq, "dk": dk, "dv": dv}
 
 
 def decode_problems(q, k, v, pairs):

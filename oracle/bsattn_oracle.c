@@ -445,3 +445,120 @@ int oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     }
     return ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------------
+ * Prefill backward, for sparsity-aware training ("BLASST: Dynamic Blocked
+ * Attention Sparsity via Softmax Thresholding", section 3.3: fine-tuning runs
+ * the forward with the skip, and the blocks it skipped receive no gradient
+ * because they were never computed).  With the forward's executed tiles held
+ * fixed (the skip decisions are piecewise constant in the inputs), O is the
+ * exact softmax over the keys of those tiles, so the gradient is that of
+ * softmax attention restricted to them.  Per query row r, over its executed,
+ * unmasked keys c:
+ *   S_rc = scale <q_r, k_c>,  P_rc = exp(S_rc - max_c S) / sum_c exp(...)
+ *   dV_c += P_rc dO_r
+ *   dP_rc = <dO_r, v_c>,  D_r = sum_c P_rc dP_rc
+ *   dS_rc = P_rc (dP_rc - D_r)
+ *   dQ_r = scale sum_c dS_rc k_c,  dK_c += scale dS_rc q_r
+ * dK and dV of a KV head sum over the query heads that read it (GQA).
+ *
+ * q, dout: [B][Hq][N][d]; k, v: [B][Hkv][N][d] (doubles).
+ * tile_status: [B][Hq][nq][nk] as the forward wrote it; only tiles marked 2
+ *   (executed) take part.  Causal and key-padding masks apply inside them.
+ * seq_lens: NULL or [B] valid lengths; padding query rows get dQ = 0.
+ * dq: [B][Hq][N][d]; dk, dv: [B][Hkv][N][d]; all overwritten.
+ */
+int oracle_prefill_bwd(const double *q, const double *k, const double *v, const double *dout,
+                       int B, int Hq, int Hkv, int N, int d, int block, double scale,
+                       int causal, const uint8_t *tile_status, const int32_t *seq_lens,
+                       double *dq, double *dk, double *dv)
+{
+    if (!q || !k || !v || !dout || !tile_status || !dq || !dk || !dv || B < 1 || Hq < 1 ||
+        Hkv < 1 || Hq % Hkv != 0 || N < 1 || d < 1 || block < 1)
+        return ORACLE_ERR_ARG;
+    if (seq_lens)
+        for (int b = 0; b < B; ++b)
+            if (seq_lens[b] < 0 || seq_lens[b] > N)
+                return ORACLE_ERR_ARG;
+    const int g = Hq / Hkv;
+    const int nq = (N + block - 1) / block, nk = nq;
+
+    /* one (sequence, KV head) per task: its dK, dV and its group's dQ */
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t w = 0; w < (int64_t)B * Hkv; ++w) {
+        const int b = (int)(w / Hkv), kvh = (int)(w % Hkv);
+        const int64_t len = seq_lens ? seq_lens[b] : N;
+        const double *kb = k + w * N * d, *vb = v + w * N * d;
+        double *dkb = dk + w * N * d, *dvb = dv + w * N * d;
+        memset(dkb, 0, sizeof(double) * (size_t)N * d);
+        memset(dvb, 0, sizeof(double) * (size_t)N * d);
+        int64_t *keys = malloc(sizeof(int64_t) * (size_t)N);
+        double *p = malloc(sizeof(double) * (size_t)N);
+        double *dp = malloc(sizeof(double) * (size_t)N);
+        for (int h = kvh * g; h < (kvh + 1) * g; ++h) {
+            const int64_t bh = (int64_t)b * Hq + h;
+            for (int64_t t = 0; t < N; ++t) {
+                const double *qr = q + (bh * N + t) * d;
+                const double *dor = dout + (bh * N + t) * d;
+                double *dqr = dq + (bh * N + t) * d;
+                for (int x = 0; x < d; ++x)
+                    dqr[x] = 0.0;
+                if (t >= len)
+                    continue;                  /* padding query row */
+                const int i = (int)(t / block);
+                const uint8_t *st = tile_status + (bh * nq + i) * nk;
+                /* the row's keys: in executed tiles, valid, not after it */
+                int nkeys = 0;
+                for (int j = 0; j < nk; ++j) {
+                    if (st[j] != 2)
+                        continue;
+                    for (int64_t c = (int64_t)j * block; c < (int64_t)(j + 1) * block; ++c)
+                        if (c < len && !(causal && c > t))
+                            keys[nkeys++] = c;
+                }
+                if (nkeys == 0)
+                    continue;
+                /* P: the softmax of the row's scores over those keys */
+                double mu = -INFINITY;
+                for (int a = 0; a < nkeys; ++a) {
+                    double acc = 0.0;
+                    for (int x = 0; x < d; ++x)
+                        acc += qr[x] * kb[keys[a] * d + x];
+                    p[a] = scale * acc;
+                    if (p[a] > mu)
+                        mu = p[a];
+                }
+                double z = 0.0;
+                for (int a = 0; a < nkeys; ++a) {
+                    p[a] = exp(p[a] - mu);
+                    z += p[a];
+                }
+                for (int a = 0; a < nkeys; ++a)
+                    p[a] /= z;
+                /* dP and D */
+                double D = 0.0;
+                for (int a = 0; a < nkeys; ++a) {
+                    double acc = 0.0;
+                    for (int x = 0; x < d; ++x)
+                        acc += dor[x] * vb[keys[a] * d + x];
+                    dp[a] = acc;
+                    D += p[a] * acc;
+                }
+                /* dS, then the three gradients */
+                for (int a = 0; a < nkeys; ++a) {
+                    const double ds = p[a] * (dp[a] - D);
+                    const int64_t c = keys[a];
+                    for (int x = 0; x < d; ++x) {
+                        dqr[x] += scale * ds * kb[c * d + x];
+                        dkb[c * d + x] += scale * ds * qr[x];
+                        dvb[c * d + x] += p[a] * dor[x];
+                    }
+                }
+            }
+        }
+        free(keys);
+        free(p);
+        free(dp);
+    }
+    return ORACLE_OK;
+}

@@ -11,6 +11,7 @@ import pytest
 import oracle
 from tests import test_oracle_pins as pins
 from tests import test_golden as golden
+from tests import test_oracle_bwd_pins as bwd
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "bsattn_oracle.c")
 
@@ -36,6 +37,18 @@ MUTANTS = {
                                  "query_tile(qrows, qpos, nrows, kb, vb, N, d,")],
     "decode_splits_cut_full_cache": [("const int chunk = Tp > 0 ? (Tp + num_splits - 1) / num_splits : 1;",
                                       "const int chunk = (T + num_splits - 1) / num_splits;")],
+    # backward
+    "bwd_drops_row_term": [("const double ds = p[a] * (dp[a] - D);", "const double ds = p[a] * dp[a];")],
+    "bwd_dk_from_keys": [("dkb[c * d + x] += scale * ds * qr[x];",
+                          "dkb[c * d + x] += scale * ds * kb[c * d + x];")],
+    "bwd_dv_from_ds": [("dvb[c * d + x] += p[a] * dor[x];", "dvb[c * d + x] += ds * dor[x];")],
+    "bwd_dq_unscaled": [("dqr[x] += scale * ds * kb[c * d + x];", "dqr[x] += ds * kb[c * d + x];")],
+    "bwd_skipped_tiles_get_gradient": [("if (st[j] != 2)", "if (st[j] == 0)")],
+    "bwd_causal_ignored": [("if (c < len && !(causal && c > t))", "if (c < len)")],
+    "bwd_unnormalised_p": [("p[a] /= z;", "(void)z;")],
+    "bwd_group_by_modulo": [("for (int h = kvh * g; h < (kvh + 1) * g; ++h)",
+                             "for (int h = kvh; h < Hq; h += Hkv)")],
+    "bwd_padding_keys_kept": [("if (c < len && !(causal && c > t))", "if (c < N && !(causal && c > t))")],
 }
 
 CHECKS = [
@@ -54,6 +67,12 @@ CHECKS = [
     pins.test_decode_gqa_group_vote,
     pins.test_index_matches_definition_and_causal,
     golden.test_causal_dense_count,
+    lambda: bwd.test_bwd_dense_equals_autograd(2, 4, 2, 200, 64, 64, True),
+    bwd.test_bwd_blasst_equals_autograd_over_executed_tiles,
+    lambda: bwd.test_bwd_central_differences_with_skips("k"),
+    bwd.test_bwd_never_executed_keys_get_no_gradient,
+    bwd.test_bwd_gqa_equals_group_sum_of_mha,
+    lambda: bwd.test_bwd_varlen_equals_each_sequence_alone(False),
 ]
 
 
