@@ -16,6 +16,7 @@
 // copied out.  Both internal streams and a ring of events are created once
 // per device and reused.  One cudaMemcpyAsync per tensor slice; host buffers
 // must be page-locked for the copies to overlap.
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -67,13 +68,23 @@ int bsattn_fwd_prefill_host(const void* h_q, const void* h_k, const void* h_v, v
                             const int32_t* row_ptr, const int32_t* col_idx,
                             const int32_t* row_order, int mask_heads, int kv_heads_per_chunk,
                             int32_t* d_status, cudaStream_t stream) {
+  // every check a chunk's bsattn_fwd_prefill would make, before any copy is
+  // enqueued, so that a rejected call leaves nothing running
   if (!h_q || !h_k || !h_v || !h_o || !d_q || !d_k || !d_v || !d_o)
     return BSATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0) return BSATTN_ERR_INVALID_ARG;
   if (kv_heads_per_chunk < 1 || Hkv % kv_heads_per_chunk != 0) return BSATTN_ERR_INVALID_ARG;
-  if (row_ptr && mask_heads != 1 && mask_heads != Hq) return BSATTN_ERR_INVALID_ARG;
+  if (!(lambda >= 0.f && lambda <= 1.f) || !std::isfinite(scale) || !(scale > 0.f))
+    return BSATTN_ERR_INVALID_ARG;
+  if (row_order && !row_ptr) return BSATTN_ERR_INVALID_ARG;
+  if (row_ptr && (!col_idx || (mask_heads != 1 && mask_heads != Hq)))
+    return BSATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return BSATTN_ERR_UNSUPPORTED;
   if (block != 64 && block != 128) return BSATTN_ERR_UNSUPPORTED;
+  // chunk offsets are multiples of N * d * 2 bytes, so aligned bases suffice
+  for (const void* ptr : {static_cast<const void*>(d_q), static_cast<const void*>(d_k),
+                          static_cast<const void*>(d_v), static_cast<const void*>(d_o)})
+    if (reinterpret_cast<uintptr_t>(ptr) & 15u) return BSATTN_ERR_ALIGNMENT;
   HostPipe* pipe = pipe_for_current_device();
   if (!pipe) return BSATTN_ERR_CUDA;
 

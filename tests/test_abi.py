@@ -121,14 +121,24 @@ def test_host_pipeline_validation(lib):
     """bsattn_fwd_prefill_host rejects bad arguments before touching a device."""
     f = lib.bsattn_fwd_prefill_host
 
-    def call(chunk=1, d=128, hq=0x1000):
-        return f(P(hq) if hq else None, P(0x2000), P(0x3000), P(0x4000), P(0x5000), P(0x6000),
-                 P(0x7000), P(0x8000), 1, 8, 2, 256, d, 128, ctypes.c_float(0.1), 1,
-                 ctypes.c_float(0.0), None, None, None, 1, chunk, None, None)
+    def call(chunk=1, d=128, hq=0x1000, dq=0x5000, do=0x8000, lam=0.0, scale=0.1, rp=None,
+             ci=None, ro=None, mh=1):
+        return f(P(hq) if hq else None, P(0x2000), P(0x3000), P(0x4000), P(dq), P(0x6000),
+                 P(0x7000), P(do), 1, 8, 2, 256, d, 128, ctypes.c_float(scale), 1,
+                 ctypes.c_float(lam), P(rp) if rp else None, P(ci) if ci else None,
+                 P(ro) if ro else None, mh, chunk, None, None)
     assert call(hq=0) == -1
     assert call(chunk=0) == -1
     assert call(chunk=3) == -1          # does not divide the two KV heads
+    assert call(lam=1.5) == -1
+    assert call(lam=float("nan")) == -1
+    assert call(scale=0.0) == -1
+    assert call(rp=0x9000) == -1        # CSR without col_idx
+    assert call(rp=0x9000, ci=0xa000, mh=3) == -1
+    assert call(ro=0xb000) == -1        # row order without a CSR
     assert call(d=96) == -2
+    assert call(dq=0x5008) == -3        # staging buffers must be 16-byte aligned
+    assert call(do=0x8004) == -3
 
 
 def test_index_host_validation(lib):
