@@ -107,8 +107,13 @@ int bsattn_debug_set(long long wait_limit_ns, int inject_stall) {
 }
 
 int bsattn_debug_trace(int n, int32_t** host_view) {
-  static int32_t* host_buf = nullptr;
   if (n < 0 || (n > 0 && !host_view)) return BSATTN_ERR_INVALID_ARG;
+#ifndef BSATTN_TRACE
+  // the shipped library has no trace markers compiled in and allocates nothing
+  if (host_view) *host_view = nullptr;
+  return n == 0 ? BSATTN_OK : BSATTN_ERR_UNSUPPORTED;
+#else
+  static int32_t* host_buf = nullptr;
   g_trace = nullptr;
   g_trace_n = 0;
   if (host_buf) {
@@ -133,6 +138,7 @@ int bsattn_debug_trace(int n, int32_t** host_view) {
   g_trace_n = n;
   *host_view = host_buf;
   return BSATTN_OK;
+#endif
 }
 
 int bsattn_build_index(const uint8_t* d_mask, int mask_heads, int nq_blocks, int nk_blocks,

@@ -25,7 +25,9 @@
 //               slot B's, so the tensor core works on one slot while the other
 //               slot's softmax runs.
 //   warps 4..7  softmax of slot A, warps 8..11 softmax of slot B: one thread
-//               per query row (TMEM lane), vote across the four warps of the slot.
+//               per query row (TMEM lane); the slot's skip decision is one
+//               barrier reduction (bar.red.and) over its four warps.  With
+//               lambda = 0 a variant compiled without the vote runs.
 //   warp 2      with V skipping only: the V producer (warp 3 idles).  The section on the
 //               prefill kernel keeps every V load (the decision comes too late
 //               to hide a conditional load's latency); as an option, a slot's
@@ -83,17 +85,15 @@ struct PairBarriers {
   uint64_t s_full[2];       // per head
   uint64_t p_ready[2];      // per head
   uint64_t o_done[2];       // per head
-  uint64_t vote_bar[2][2];  // per head, tile parity
   uint64_t dq_full[2][4], dq_empty[2][4];   // per slot: decisions to the V producer
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
   int skip_flag[2];
-  int vote[2][2][4];        // head, tile parity, warp
   int dval[2][4];           // 1 = kept
 };
 
-template <int D, bool SKIPV>
+template <int D, bool SKIPV, bool VOTE>
 __global__ void __launch_bounds__(384, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
@@ -213,8 +213,6 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->s_full[s], 1);
       mbar_init(&bars->p_ready[s], 4);
       mbar_init(&bars->o_done[s], 1);
-      mbar_init(&bars->vote_bar[s][0], 4);
-      mbar_init(&bars->vote_bar[s][1], 4);
       for (int x = 0; x < C::DQ; ++x) {
         mbar_init(&bars->dq_full[s][x], 1);
         mbar_init(&bars->dq_empty[s][x], 1);
@@ -364,9 +362,16 @@ __global__ void __launch_bounds__(384, 1)
   #pragma unroll
           for (int e = 0; e < 2; ++e) {
             if (t >= tb[e] && t < te[e]) {   // this slot takes part in step t
-              if (!mbar_wait(&bars->p_ready[e], (t - tb[e]) & 1, abort, lim)) { ok = false; break; }
-              tc_fence_after();
-              const int skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[e]);
+              int skip = 0;
+              if (VOTE) {
+                if (!mbar_wait(&bars->p_ready[e], (t - tb[e]) & 1, abort, lim)) { ok = false; break; }
+                tc_fence_after();
+                skip = *reinterpret_cast<volatile int*>(&bars->skip_flag[e]);
+              } else {
+                // no skipping: every tile is kept and p_ready completes once per tile
+                if (!mbar_wait(&bars->p_ready[e], kept[e] & 1, abort, lim)) { ok = false; break; }
+                tc_fence_after();
+              }
               if (!skip) {
                 if (!v_ready) {
                   if (!mbar_wait(&bars->v_full[vs], (vi / C::VST) & 1, abort, lim)) { ok = false; break; }
@@ -432,9 +437,14 @@ __global__ void __launch_bounds__(384, 1)
       for (int t = 0; t < ne; ++t) {       // t counts this slot's tiles
         const int u = u0 + du * t;
         const int j = cols ? cols[u] : u;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[e], t & 1, abort, lim))) {
+        // A warp whose wait ran out (ok false) does no more work, but it still
+        // meets the slot's other warps at the vote barrier once per tile, so
+        // no warp is ever left waiting there: nothing in the loop leaves it
+        // early.
+        if (!ok || !__all_sync(0xffffffffu, mbar_wait(&bars->s_full[e], t & 1, abort, lim))) {
           ok = false;
-          break;
+          if (VOTE) bar_red_and(1 + e, 128, true);
+          continue;
         }
         tc_fence_after();
         uint32_t r[BLK];
@@ -451,24 +461,13 @@ __global__ void __launch_bounds__(384, 1)
             if (key >= lenb || (p.causal && key > qpos)) r[c] = __float_as_uint(-INFINITY);
           }
         }
-        const float mx = row_max<BLK>(reinterpret_cast<const float*>(r));
-        const float mt = mx * p.scale_log2;
+        const float mt = row_max<BLK>(reinterpret_cast<const float*>(r)) * p.scale_log2;
         int skip = 0;
-        if (p.use_skip) {
+        if (VOTE) {
+          // the slot's decision: every valid row of the query tile passes.  One
+          // barrier reduction over the slot's four warps (named barrier 1 + e)
           const bool pass = !valid || (mt - m_run < p.thr_log2);
-          const bool wpass = __all_sync(0xffffffffu, pass);
-          if (lane == 0) {
-            bars->vote[e][t & 1][sw] = wpass ? 1 : 0;
-            mbar_arrive(&bars->vote_bar[e][t & 1]);
-          }
-          __syncwarp();
-          if (!__all_sync(0xffffffffu,
-                          mbar_wait(&bars->vote_bar[e][t & 1], (t >> 1) & 1, abort, lim))) {
-            ok = false;
-            break;
-          }
-          volatile int* vv = bars->vote[e][t & 1];
-          skip = vv[0] & vv[1] & vv[2] & vv[3];
+          skip = bar_red_and(1 + e, 128, pass) ? 1 : 0;
         }
         if (SKIPV) {   // the decision to the V producer, before any exponential
           if (sw == 0 && lane == 0) {
@@ -480,7 +479,7 @@ __global__ void __launch_bounds__(384, 1)
           }
           if (__any_sync(0xffffffffu, *abort != 0)) {
             ok = false;
-            break;
+            continue;
           }
         }
         m_run = fmaxf(m_run, mt);
@@ -492,7 +491,7 @@ __global__ void __launch_bounds__(384, 1)
             // reading P; wait for it to land in O before O may be rescaled
             if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done[e], (kept - 1) & 1, abort, lim))) {
               ok = false;
-              break;
+              continue;
             }
             tc_fence_after();
           }
@@ -541,7 +540,7 @@ __global__ void __launch_bounds__(384, 1)
           tmem_wait_st();
           ++kept;
         }
-        if (sw == 0 && lane == 0) bars->skip_flag[e] = skip;
+        if (VOTE && sw == 0 && lane == 0) bars->skip_flag[e] = skip;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->p_ready[e]);
@@ -594,13 +593,13 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int D, bool SKIPV>
+template <int D, bool SKIPV, bool VOTE>
 static cudaError_t launch_pair(const CUtensorMap& tq, const CUtensorMap& tk,
                                const CUtensorMap& tv, const PrefillParams& p, int grid,
                                cudaStream_t stream) {
   using C = PairCfg<D>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(prefill_pair_kernel<D, SKIPV>,
+  cudaError_t e = cudaFuncSetAttribute(prefill_pair_kernel<D, SKIPV, VOTE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   static_assert(128 * C::REG_LOW + 256 * C::REG_HIGH == C::THREADS * C::REG_LAUNCH,
@@ -608,10 +607,10 @@ static cudaError_t launch_pair(const CUtensorMap& tq, const CUtensorMap& tk,
   // setmaxnreg.inc waits until the block's pool has the registers; launch only
   // when the compiled kernel reserves the REG_LAUNCH the split is built on
   cudaFuncAttributes attr;
-  e = cudaFuncGetAttributes(&attr, prefill_pair_kernel<D, SKIPV>);
+  e = cudaFuncGetAttributes(&attr, prefill_pair_kernel<D, SKIPV, VOTE>);
   if (e != cudaSuccess) return e;
   if (attr.numRegs != C::REG_LAUNCH) return cudaErrorInvalidConfiguration;
-  prefill_pair_kernel<D, SKIPV><<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
+  prefill_pair_kernel<D, SKIPV, VOTE><<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -619,8 +618,11 @@ template <int D>
 cudaError_t launch_prefill_pair(const CUtensorMap& tq, const CUtensorMap& tk,
                                 const CUtensorMap& tv, const PrefillParams& p, int grid,
                                 cudaStream_t stream) {
-  return p.skip_v ? launch_pair<D, true>(tq, tk, tv, p, grid, stream)
-                  : launch_pair<D, false>(tq, tk, tv, p, grid, stream);
+  // lambda = 0: a kernel without the vote (nothing is skipped, so V skipping
+  // has nothing to skip either)
+  if (!p.use_skip) return launch_pair<D, false, false>(tq, tk, tv, p, grid, stream);
+  return p.skip_v ? launch_pair<D, true, true>(tq, tk, tv, p, grid, stream)
+                  : launch_pair<D, false, true>(tq, tk, tv, p, grid, stream);
 }
 
 template cudaError_t launch_prefill_pair<128>(const CUtensorMap&, const CUtensorMap&,

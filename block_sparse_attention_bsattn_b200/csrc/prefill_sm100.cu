@@ -418,14 +418,9 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
       if (sw == 0 && lane == 0 && p.tile_status && (unsigned)j < (unsigned)p.nk)
         p.tile_status[(((int64_t)b * p.Hq + h) * p.nq + i) * p.nk + j] = skip ? 1 : 2;
       if (!skip) {
-        if (kept > 0) {
-          // the previous BMM2 must be complete before O may be rescaled
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (kept - 1) & 1, abort, lim))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-        }
+        // P of this tile goes to the other S buffer than the one the previous
+        // kept tile's BMM2 may still be reading, so the exponentials need not
+        // wait for that BMM2; only a rescale of O does (below).
         // exponent shift: set by the first kept tile, then moved only when the
         // running max exceeds it by more than TAU (O and l rescaled below);
         // both halves of a row compute the same shift
@@ -459,8 +454,17 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
           const float2 rs2 = fadd2(fadd2(rs4[0], rs4[1]), fadd2(rs4[2], rs4[3]));
           const float rs = rs2.x + rs2.y;
           l = l * alpha + rs;
-          // rare: bring this half of the accumulated O to the new shift
+          // rare: bring this half of the accumulated O to the new shift, once
+          // every earlier kept tile's BMM2 has landed in it.  The wait is for
+          // the newest BMM2 that can have been issued (this tile's needs this
+          // warp's hand-over), so skipping the waits of earlier phases cannot
+          // confuse the phase parity.
           if (__any_sync(0xffffffffu, rescale)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (kept - 1) & 1, abort, lim))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
 #pragma unroll
             for (int c0 = 0; c0 < OW; c0 += 32) {
               uint32_t ro[32];

@@ -238,6 +238,23 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// AND of `pred` over the `nthreads` threads (whole warps) that meet at named
+// barrier `id`; every one of them gets the result.  A hardware barrier has no
+// time limit, so callers must make every participating warp reach it the same
+// number of times, whatever happens to their other waits.
+__device__ __forceinline__ bool bar_red_and(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -308,15 +325,20 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// Debug progress marker: slot `i` (< 1024) of a host-visible trace buffer
-// (no-op when tracing is off).  Stores are volatile and fenced at system scope
-// so that a host thread can watch them while the kernel runs.
+// Debug progress marker: slot `i` (< 1024) of a host-visible trace buffer.
+// Compiled only into a debugging build (-DBSATTN_TRACE); in the shipped
+// library it is empty and costs nothing.  Stores are volatile and fenced at
+// system scope so that a host thread can watch them while the kernel runs.
+#ifdef BSATTN_TRACE
 __device__ __forceinline__ void trace_mark(volatile int32_t* trace, int n, int i, int32_t v) {
   if (trace && i < n && i < 1024) {
     trace[i] = v;
     __threadfence_system();
   }
 }
+#else
+__device__ __forceinline__ void trace_mark(volatile int32_t*, int, int, int32_t) {}
+#endif
 
 __device__ __forceinline__ void report_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, 0, code);

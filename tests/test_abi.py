@@ -155,3 +155,13 @@ def test_index_host_validation(lib):
 def test_debug_hook_validation(lib):
     assert lib.bsattn_debug_set(0, 0) == -1
     assert lib.bsattn_debug_set(2_000_000_000, 0) == 0
+
+
+def test_shipped_library_has_no_trace_buffer(lib):
+    """The trace markers are a debugging build's (-DBSATTN_TRACE): the shipped
+    library refuses to allocate a trace buffer and accepts turning it off."""
+    view = ctypes.POINTER(ctypes.c_int32)()
+    assert lib.bsattn_debug_trace(16, ctypes.byref(view)) == -2   # BSATTN_ERR_UNSUPPORTED
+    assert not view
+    assert lib.bsattn_debug_trace(0, None) == 0
+    assert lib.bsattn_debug_trace(-1, None) == -1
