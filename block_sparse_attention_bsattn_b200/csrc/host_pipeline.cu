@@ -85,8 +85,28 @@ int bsattn_fwd_prefill_host(const void* h_q, const void* h_k, const void* h_v, v
   for (const void* ptr : {static_cast<const void*>(d_q), static_cast<const void*>(d_k),
                           static_cast<const void*>(d_v), static_cast<const void*>(d_o)})
     if (reinterpret_cast<uintptr_t>(ptr) & 15u) return BSATTN_ERR_ALIGNMENT;
+  {
+    // the chunks' kernels need compute capability 10.x: refuse before any copy
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return BSATTN_ERR_CUDA;
+    if (major != 10) return BSATTN_ERR_UNSUPPORTED;
+  }
+  const int64_t nq_all = (N + block - 1) / block;
+  if ((int64_t)(Hq / Hkv) * kv_heads_per_chunk * nq_all > INT32_MAX) return BSATTN_ERR_UNSUPPORTED;
   HostPipe* pipe = pipe_for_current_device();
   if (!pipe) return BSATTN_ERR_CUDA;
+  // On a failure part-way, the caller's stream is still made to wait for
+  // everything already queued on the internal streams (copies and kernels that
+  // read or write the caller's buffers) before the error is returned.
+  auto fail = [&](int rc) {
+    if (cudaEventRecord(pipe->done, pipe->in) == cudaSuccess)
+      cudaStreamWaitEvent(stream, pipe->done, 0);
+    if (cudaEventRecord(pipe->done, pipe->out) == cudaSuccess)
+      cudaStreamWaitEvent(stream, pipe->done, 0);
+    return rc;
+  };
 
   const int G = Hq / Hkv;
   const int hkc = kv_heads_per_chunk, hqc = hkc * G;     // heads per chunk
@@ -101,7 +121,7 @@ int bsattn_fwd_prefill_host(const void* h_q, const void* h_k, const void* h_v, v
   if (cudaEventRecord(pipe->start, stream) != cudaSuccess ||
       cudaStreamWaitEvent(pipe->in, pipe->start, 0) != cudaSuccess ||
       cudaStreamWaitEvent(pipe->out, pipe->start, 0) != cudaSuccess)
-    return BSATTN_ERR_CUDA;
+    return fail(BSATTN_ERR_CUDA);
 
   int c = 0;
   for (int b = 0; b < B; ++b) {
@@ -118,7 +138,7 @@ int bsattn_fwd_prefill_host(const void* h_q, const void* h_k, const void* h_v, v
                           pipe->in) != cudaSuccess ||
           cudaEventRecord(copied, pipe->in) != cudaSuccess ||
           cudaStreamWaitEvent(stream, copied, 0) != cudaSuccess)
-        return BSATTN_ERR_CUDA;
+        return fail(BSATTN_ERR_CUDA);
       // the chunk as a problem of its own: one sequence, hqc query heads;
       // per-head CSR rows and orders start at the chunk's first head
       const bool per_head = row_ptr && mask_heads == Hq;
@@ -128,12 +148,12 @@ int bsattn_fwd_prefill_host(const void* h_q, const void* h_k, const void* h_v, v
           row_ptr ? row_ptr + (per_head ? (size_t)hq0 * (nq + 1) : 0) : nullptr, col_idx,
           row_order ? row_order + (per_head ? (size_t)hq0 * nq : 0) : nullptr,
           per_head ? hqc : 1, nullptr, d_status, stream);
-      if (rc != BSATTN_OK) return rc;
+      if (rc != BSATTN_OK) return fail(rc);
       if (cudaEventRecord(computed, stream) != cudaSuccess ||
           cudaStreamWaitEvent(pipe->out, computed, 0) != cudaSuccess ||
           cudaMemcpyAsync(atw(h_o, qoff), at(d_o, qoff), qlen, cudaMemcpyDeviceToHost,
                           pipe->out) != cudaSuccess)
-        return BSATTN_ERR_CUDA;
+        return fail(BSATTN_ERR_CUDA);
     }
   }
   // the caller's stream completes after the last copy out

@@ -96,9 +96,12 @@ def bsattn_debug_set(wait_limit_ns: int = 2_000_000_000, inject_stall: bool = Fa
 
 
 def bsattn_debug_trace(n: int):
-    """Debugging aid: n > 0 makes the kernels record progress markers into a
-    library-owned mapped host buffer of n int32 and returns a numpy view of it
-    (readable while a kernel runs); n = 0 turns tracing off and returns None."""
+    """Debugging aid of a library built with -DBSATTN_TRACE: n > 0 makes the
+    kernels record progress markers into a library-owned mapped host buffer of
+    n int32 and returns a numpy view of it (readable while a kernel runs);
+    n = 0 turns tracing off and returns None.  The shipped library has no
+    markers compiled in and raises BsattnError(BSATTN_ERR_UNSUPPORTED) for
+    n > 0."""
     import numpy as np
     view = ctypes.POINTER(ctypes.c_int32)()
     rc = _lib.bsattn_debug_trace(int(n), ctypes.byref(view))
@@ -120,6 +123,20 @@ def _check(t: torch.Tensor, name: str, dtype, dims: int):
     if not isinstance(t, torch.Tensor) or t.dtype != dtype or t.dim() != dims or not t.is_cuda \
             or not t.is_contiguous():
         raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor with {dims} dims")
+
+
+def _check_buf(t: Optional[torch.Tensor], name: str, dtype, numel: int, exact: bool = False):
+    """A caller-supplied output buffer: contiguous CUDA `dtype`, holding at
+    least (or, with `exact`, exactly) `numel` elements, so that no kernel
+    writes past its end."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or not t.is_cuda \
+            or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor")
+    if (t.numel() != numel) if exact else (t.numel() < numel):
+        raise ValueError(f"{name}: {'exactly' if exact else 'at least'} {numel} elements "
+                         f"needed, got {t.numel()}")
 
 
 def bsattn_build_index(mask: torch.Tensor, q_block: int, k_block: int, causal: bool = False,
@@ -173,6 +190,11 @@ def bsattn_fwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
         raise ValueError("k/v must be [B, Hkv, N, d] matching q")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    nq = -(-N // int(block))
+    _check_buf(o, "o", torch.bfloat16, B * Hq * N * d, exact=True)
+    _check_buf(lse, "lse", torch.float32, B * Hq * N, exact=True)
+    _check_buf(tile_status, "tile_status", torch.uint8, B * Hq * nq * nq)
+    _check_buf(status, "status", torch.int32, 1)
     if o is None:
         o = torch.empty_like(q)
     if lse is None and want_lse:
@@ -233,6 +255,14 @@ def bsattn_decode_workspace_size(B: int, Hq: int, d: int, num_splits: int) -> in
     return int(_lib.bsattn_decode_workspace_size(B, Hq, d, num_splits))
 
 
+def _check_decode_bufs(B, Hq, Hkv, L, d, block, o, lse, tile_status, status):
+    T = -(-L // int(block))
+    _check_buf(o, "o", torch.bfloat16, B * Hq * d, exact=True)
+    _check_buf(lse, "lse", torch.float32, B * Hq, exact=True)
+    _check_buf(tile_status, "tile_status", torch.uint8, B * Hkv * T)
+    _check_buf(status, "status", torch.int32, 1)
+
+
 def bsattn_fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int,
                       num_splits: int, scale: Optional[float] = None, lam: float = 0.0,
                       o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
@@ -253,6 +283,7 @@ def bsattn_fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: 
         raise ValueError("k/v must be [B, Hkv, L, d] matching q")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    _check_decode_bufs(B, Hq, Hkv, L, d, block, o, lse, tile_status, status)
     if o is None:
         o = torch.empty_like(q)
     if lse is None and want_lse:
@@ -260,6 +291,8 @@ def bsattn_fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: 
     need = bsattn_decode_workspace_size(B, Hq, d, num_splits)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    elif not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace: expected a contiguous CUDA tensor")
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, L, d, int(block),
             float(scale), 0, float(lam), int(num_splits), _ptr(workspace),
             workspace.numel() * workspace.element_size(), _ptr(tile_status))
@@ -295,6 +328,7 @@ def bsattn_fwd_decode_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         raise ValueError("k/v must be [B, Hkv, L, d] and o [B, Hq, d] matching q")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    _check_decode_bufs(B, Hq, Hkv, L, d, block, o, lse, tile_status, status)
     rc = _lib.bsattn_fwd_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq,
                                         Hkv, L, d, int(block), float(scale), 0, float(lam),
                                         int(num_splits), _ptr(tile_status), _ptr(status),

@@ -22,9 +22,12 @@
  *  - GQA ("Attention 的七十二变", section 5.3-5.4): query head h reads KV head
  *    h / (Hq / Hkv).
  *  - All pointers are device pointers unless stated otherwise.  The caller
- *    allocates and owns every buffer; the library allocates no device memory
- *    and keeps no state between calls besides a per-device cache of kernel
- *    attributes.
+ *    allocates and owns every buffer; no call allocates device memory.  One
+ *    fixed reservation comes with the library itself: loading it places the
+ *    32 MiB scratch array of bsattn_fwd_decode_noalloc on every device that
+ *    uses the library, for the life of the process.  Between calls the
+ *    library keeps only per-device caches (kernel attributes, the host-buffer
+ *    prefill's streams and events, the scratch array's address).
  *  - Every call is asynchronous on `stream`.  The return value reports only
  *    host-side validation and launch errors; nothing is launched when it is
  *    not BSATTN_OK.  Errors found on the device (a pipeline wait that ran out
@@ -72,16 +75,19 @@ int bsattn_version(void);
 int bsattn_debug_set(long long wait_limit_ns, int inject_stall);
 
 /*
- * bsattn_debug_trace -- debugging aid, process-wide.  n > 0 allocates n int32
- * of mapped, pinned host memory (zeroed; the only allocation the library ever
- * makes, and on the host), returns its host address in *host_view and makes
- * the prefill and decode kernels record progress there, readable while a
- * kernel is still running: slot 16 + CTA index holds the stage a CTA reached
+ * bsattn_debug_trace -- debugging aid, process-wide, present only in a
+ * library built with -DBSATTN_TRACE.  The shipped library has no trace
+ * markers compiled into its kernels: there n = 0 returns BSATTN_OK (and sets
+ * *host_view to NULL when given), n > 0 returns BSATTN_ERR_UNSUPPORTED and
+ * allocates nothing.  In a trace build, n > 0 allocates n int32 of mapped,
+ * pinned host memory (zeroed), returns its host address in *host_view and
+ * makes the prefill and decode kernels record progress there, readable while
+ * a kernel is still running: slot 16 + CTA index holds the stage a CTA reached
  * (1 entered, 2 set up, 3 finished, 4 tensor memory freed; 13/14 the same
  * after a timed-out wait), slots 8..17 the warps of CTA 0 that have left
- * their role's loop (one-query-tile prefill kernel).  n = 0
- * frees the buffer and turns tracing off.  Negative n or a NULL host_view
- * with n > 0 give BSATTN_ERR_INVALID_ARG.
+ * their role's loop (one-query-tile prefill kernel); n = 0 frees the buffer
+ * and turns tracing off.  Negative n or a NULL host_view with n > 0 give
+ * BSATTN_ERR_INVALID_ARG in both builds.
  */
 int bsattn_debug_trace(int n, int32_t **host_view);
 
@@ -211,7 +217,11 @@ int bsattn_fwd_prefill_ex(const void *q, const void *k, const void *v, void *o, 
  * completes.  The first call on a device creates two streams and a ring of
  * events for it, kept until the process exits.  No LSE or tile status is
  * produced.  Errors as in bsattn_fwd_prefill, plus BSATTN_ERR_INVALID_ARG for
- * a chunk size that does not divide Hkv.
+ * a chunk size that does not divide Hkv.  Every argument check (and the
+ * compute-capability check) comes before any copy is enqueued.  If a later
+ * step fails part-way (a copy or a chunk's launch), `stream` is still made to
+ * wait for everything already queued on the internal streams before the error
+ * is returned, so the caller may reuse its buffers once `stream` completes.
  */
 int bsattn_fwd_prefill_host(const void *h_q, const void *h_k, const void *h_v, void *h_o,
                             void *d_q, void *d_k, void *d_v, void *d_o, int B, int Hq, int Hkv,
@@ -298,15 +308,20 @@ int bsattn_fwd_decode_ex(const void *q, const void *k, const void *v, void *o, f
  * until the process exits.  The call itself allocates nothing.
  *
  * Arguments, layouts and results are those of bsattn_fwd_decode without the
- * workspace.  Problems whose split outputs need more than 32 MiB
- * (bsattn_decode_workspace_size(B, Hq, d, num_splits) > 33554432) are rejected
- * with BSATTN_ERR_CAPACITY before anything runs.
+ * workspace.  Checks come in this order: NULL q/k/v/o, non-positive sizes or
+ * Hq % Hkv != 0 give BSATTN_ERR_INVALID_ARG; then problems whose split
+ * outputs need more than 32 MiB (bsattn_decode_workspace_size(B, Hq, d,
+ * num_splits) > 33554432) give BSATTN_ERR_CAPACITY; then every other check of
+ * bsattn_fwd_decode.  Nothing runs on a rejected call.
  *
- * The first call on each device (with that device current) looks up the
- * scratch array's device address once, so make it before any stream capture.
- * Every call shares the one scratch array, which keeps the last call's
- * contents; no part of it needs to start at zero.  Calls whose kernels may
- * overlap on the GPU (unordered streams) race on it and must be serialised.
+ * The first call in each CUDA context (in practice: on each device, with that
+ * device current) looks up the scratch array's device address and caches it
+ * under the context's unique id, so make that call before any stream capture.
+ * A later context on the same device (after cudaDeviceReset) looks it up
+ * again.  Every call shares the one scratch array, which keeps the last
+ * call's contents; no part of it needs to start at zero.  Calls whose kernels
+ * may overlap on the GPU (unordered streams) race on it and must be
+ * serialised.
  */
 int bsattn_fwd_decode_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
                               int B, int Hq, int Hkv, int L, int d, int block, float scale,
