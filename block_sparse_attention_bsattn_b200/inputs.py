@@ -42,6 +42,14 @@ import torch
 # prefill workload, the operating point the BLASST page reports (74.7%
 # prefill sparsity, section A1).
 SINK_BETA = 3.4
+
+# The decode operating point of the BLASST page (73.2% of V tiles skipped,
+# page summary): on the decode recipe it is reached with 4 splits of the
+# KV sequence at a = 160 (lambda = a / L), fixed once by a sweep with the CPU
+# oracle (tests/golden/calibrate_decode_operating_point.py, output in
+# tests/golden/decode_operating_point.txt).
+DECODE_OP_SPLITS = 4
+DECODE_OP_A = 160.0
 CLUSTER_TOKENS = 256
 
 

@@ -90,11 +90,13 @@ def prefill_margins(q: torch.Tensor, k: torch.Tensor, block: int, scale: float, 
 
 
 def decode_margins(q: torch.Tensor, k: torch.Tensor, block: int, scale: float,
-                   num_splits: int, pairs=None) -> np.ndarray:
+                   num_splits: int, pairs=None, sink_seed: bool = False) -> np.ndarray:
     """D for every key tile of a split-KV decode: the query tile is the GQA
     group of one token (all g rows valid), the KV tiles are cut into
     num_splits contiguous chunks of ceil(T / num_splits) tiles, and the
-    running max starts from -inf at each chunk start.
+    running max starts from -inf at each chunk start -- or, with sink_seed,
+    every chunk after the first starts from the row maxima of key tile 0 (the
+    tile of the attention sink), scored but not visited.
 
     q [B,Hq,d], k [B,Hkv,L,d].  pairs: None (every (b, kv head)) or a list
     of (b, kv head).  Returns float64 [len(pairs), T]."""
@@ -117,8 +119,10 @@ def decode_margins(q: torch.Tensor, k: torch.Tensor, block: int, scale: float,
             c1 = min(T, c0 + chunk)
             tm = tmax[:, c0:c1]
             prev = torch.cummax(tm, dim=1).values
-            mprev = torch.cat([torch.full((g, 1), -math.inf, dtype=torch.float64),
-                               prev[:, :-1]], dim=1)
+            start = torch.full((g, 1), -math.inf, dtype=torch.float64)
+            if sink_seed and c0 > 0:
+                start = tmax[:, :1].clone()
+            mprev = torch.cat([start, torch.maximum(prev[:, :-1], start)], dim=1)
             dr = tm - mprev
             dr = torch.where(torch.isnan(dr), torch.full_like(dr, math.inf), dr)
             out[p, c0:c1] = dr.amax(dim=0).numpy()

@@ -69,6 +69,24 @@ def test_decode_margins_equal_oracle_on_shrunk_blasst_decode(a):
     _same_margins(mg, ref["margin"], ref["status"] > 0)
 
 
+@pytest.mark.parametrize("a", [0.01, 1.0, 10.0])
+def test_decode_margins_sink_seed_equal_oracle(a):
+    """Sink-seeded splits: every split after the first starts its running max
+    from key tile 0's row maxima."""
+    w = inputs.workload("blasst_decode", shrink=True)
+    lam = inputs.lambda_for(a, w.N)
+    D = tile_margins.decode_margins(w.q, w.k, w.block, w.scale, w.num_splits, sink_seed=True)
+    st, mg = tile_margins.status_from_margins(D, lam)
+    pairs = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    qs, ks, vs = oracle.decode_problems(w.q, w.k, w.v, pairs)
+    ref = oracle.decode(qs, ks, vs, w.block, w.scale, lam, w.num_splits, sink_seed=True)
+    assert (st == ref["status"]).all()
+    _same_margins(mg, ref["margin"], ref["status"] > 0)
+    plain, _ = tile_margins.status_from_margins(
+        tile_margins.decode_margins(w.q, w.k, w.block, w.scale, w.num_splits), lam)
+    assert (st == 1).sum() >= (plain == 1).sum()
+
+
 def test_status_from_margins_closed_form():
     """D = NaN: not visited; lambda = 0: every visited tile executed with an
     infinite margin; otherwise skipped exactly when D < ln lambda, including
