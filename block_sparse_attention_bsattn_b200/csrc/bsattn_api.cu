@@ -240,6 +240,16 @@ int bsattn_fwd_prefill_ex(const void* q, const void* k, const void* v, void* o, 
                  : launch_prefill_pair<64>(tq, tk, tv, p, (int)pitems, stream);
     return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
   }
+  // Block masks whose rows no two query tiles share (one query head per KV
+  // head with a mask, or one mask per head): two query tiles per CTA with
+  // visit lists of their own, streamed through one ring.  V skipping keeps
+  // the one-tile kernel, which has a warp for conditional V loads.
+  if (block == 128 && !p.skip_v) {
+    const int64_t dgrid = (items + 1) / 2;
+    e = d == 128 ? launch_prefill_duo<128>(tq, tk, tv, p, (int)dgrid, stream)
+                 : launch_prefill_duo<64>(tq, tk, tv, p, (int)dgrid, stream);
+    return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+  }
   if (d == 128 && block == 128) e = launch_prefill<128, 128>(tq, tk, tv, p, (int)items, stream);
   else if (d == 64 && block == 128) e = launch_prefill<64, 128>(tq, tk, tv, p, (int)items, stream);
   else if (d == 128 && block == 64) e = launch_prefill<128, 64>(tq, tk, tv, p, (int)items, stream);

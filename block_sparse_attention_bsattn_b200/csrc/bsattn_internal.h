@@ -80,6 +80,11 @@ cudaError_t launch_prefill_pair(const CUtensorMap& tq, const CUtensorMap& tk,
                                 const CUtensorMap& tv, const PrefillParams& p, int grid,
                                 cudaStream_t stream);
 
+template <int D>
+cudaError_t launch_prefill_duo(const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const PrefillParams& p, int grid,
+                               cudaStream_t stream);
+
 template <int D, int BLK, int G>
 cudaError_t launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv,
                                 const DecodeParams& p, int grid, cudaStream_t stream);

@@ -56,6 +56,14 @@ def test_blasst_decode_shrunk(a):
     _check(w.q, w.k, w.v, w.block, w.num_splits, w.scale, inputs.lambda_for(a, w.N), what=f"a={a}")
 
 
+def test_decode_operating_point_shrunk():
+    """The benchmark's decode operating point (4 splits, a = 160: the BLASST
+    page's 73.2% decode sparsity on this recipe) on the shrunk workload."""
+    w = inputs.workload("blasst_decode", shrink=True)
+    _check(w.q, w.k, w.v, w.block, inputs.DECODE_OP_SPLITS, w.scale,
+           inputs.lambda_for(inputs.DECODE_OP_A, w.N), what="operating point")
+
+
 @pytest.mark.parametrize("d,block,g", [(64, 64, 1), (64, 128, 2), (128, 64, 8), (128, 128, 4),
                                        (128, 128, 8), (128, 128, 3), (64, 128, 16),
                                        (128, 128, 1), (128, 128, 16), (128, 128, 5),

@@ -22,23 +22,34 @@ def _ops():
 
 
 # two heads of one KV head (pair kernel, heads mode), one head (pair kernel,
-# two consecutive query tiles), 64-token tiles (one-query-tile kernel)
-@pytest.mark.parametrize("hq,hkv,block", [(2, 1, 128), (1, 1, 128), (1, 1, 64)])
-def test_stalled_pipeline_reports_timeout_and_recovers(hq, hkv, block):
+# two consecutive query tiles), 64-token tiles (one-query-tile kernel), a
+# block mask with one query head per KV head (two query tiles with visit
+# lists of their own); lambda > 0 runs the variants with the skip vote, whose
+# warps must all still meet at the vote barrier after the wait ran out
+@pytest.mark.parametrize("hq,hkv,block,masked", [(2, 1, 128, False), (1, 1, 128, False),
+                                                 (1, 1, 64, False), (2, 2, 128, True)])
+@pytest.mark.parametrize("lam", [0.0, 1e-3])
+def test_stalled_pipeline_reports_timeout_and_recovers(hq, hkv, block, masked, lam):
     ops = _ops()
     q, k, v = inputs.normal_qkv(1, hq, hkv, 256, 128, "cpu", 3)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    rp = ci = mask = None
+    if masked:
+        nb = 256 // block
+        mask = torch.ones(1, nb, nb, dtype=torch.uint8)
+        rp, ci, _ = ops.bsattn_build_index(mask.cuda(), block, block, True)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     try:
         ops.bsattn_debug_set(50_000_000, inject_stall=True)   # 50 ms per wait
-        ops.bsattn_fwd_prefill(qd, kd, vd, block, None, True, 0.0, status=status)
+        ops.bsattn_fwd_prefill(qd, kd, vd, block, None, True, lam, rp, ci, status=status)
         torch.cuda.synchronize()
         assert status.item() == -6, ops.bsattn_status_string(status.item())
     finally:
         ops.bsattn_debug_set(2_000_000_000, inject_stall=False)
     status.zero_()
-    o, lse = ops.bsattn_fwd_prefill(qd, kd, vd, block, None, True, 0.0, status=status)
+    o, lse = ops.bsattn_fwd_prefill(qd, kd, vd, block, None, True, lam, rp, ci, status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
-    ref = oracle.prefill(q, k, v, block, 1 / math.sqrt(128), True, 0.0)
+    ref = oracle.prefill(q, k, v, block, 1 / math.sqrt(128), True, lam,
+                         mask=None if mask is None else mask.numpy())
     compare_outputs(o, ref["o"], lse, ref["lse"], "after timeout")

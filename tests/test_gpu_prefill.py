@@ -368,3 +368,33 @@ def test_videodit_full_size_sampled():
 def test_blasst_prefill_full_size_sampled(a):
     w = inputs.workload("blasst_prefill", device="cuda")
     _check_sampled(w, inputs.lambda_for(a, w.N), None, 24, f"blasst a={a}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("lam", [0.0, 3e-3])
+@pytest.mark.parametrize("per_head", [False, True])
+def test_two_tile_kernel_own_lists(d, causal, lam, per_head):
+    """Masks whose rows no two query tiles share (one query head per KV head,
+    or one mask per head) run two query tiles per CTA, each with its own
+    visit list: an odd number of query tiles (the last CTA holds one), rows
+    of very different lengths, empty rows and a ragged tail."""
+    rng = np.random.default_rng(d + 2 * causal + (lam > 0) + 4 * per_head)
+    B, Hq, Hkv, N = 1, 3, 3 if not per_head else 1, 5 * 128 - 17
+    nb = -(-N // 128)
+    hm = Hq if per_head else 1
+    m = (rng.random((hm, nb, nb)) < 0.5).astype(np.uint8)
+    m[:, np.arange(nb), np.arange(nb)] = 1
+    m[:, 0, :] = 1                                 # a long row next to short ones
+    m[:, 3, :] = 0                                 # an empty row
+    q, k, v = inputs.blasst_prefill_qkv(B, Hq, Hkv, N, d, "cpu", 91 + d)
+    w = inputs.Workload("own", B, Hq, Hkv, N, d, 128, causal, "prefill", 1 / math.sqrt(d), None,
+                        q=q, k=k, v=v)
+    assert (B * Hq * nb) % 2 == 1
+    o, lse, st = _run_gpu(w, lam, m)
+    ref = oracle.prefill(q, k, v, 128, w.scale, causal, lam, mask=m)
+    compare_outputs(o, ref["o"], lse, ref["lse"], f"d{d} causal={causal} lam={lam}")
+    compare_status(st, ref["status"], ref["margin"], f"d{d} causal={causal} lam={lam}")
+    rows = slice(3 * 128, 4 * 128)
+    assert (o[:, :, rows].float() == 0).all()
+    assert torch.isneginf(lse[:, :, rows]).all()
