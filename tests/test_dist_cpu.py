@@ -1,7 +1,10 @@
 """The benchmark's multi-rank plumbing with two gloo ranks on the CPU: the
 slowest rank's time sets the step, work adds up over ranks, and every rank
 draws a different batch of the same workload (weak scaling, no collective on
-the data path)."""
+the data path).  Each rank runs the oracle on its own shard (a small BLASST
+prefill drawn with its seed); the whole job's executed tiles are the sum over
+ranks, and every rank's result equals the same shard computed in one
+process."""
 import os
 import socket
 
@@ -39,13 +42,26 @@ def _run(rank, world, port, q):
         units = bench.sum_over_ranks(100.0 * (rank + 1))
         rate = bench.whole_job_rate(100.0 * (rank + 1), 10.0 + rank)
         seeds = bench.rank_seeds(rank)
-        from block_sparse_attention_bsattn_b200 import inputs
-        # the same recipe drawn with this rank's seed (small shape, CPU)
-        qt, _, _ = inputs.blasst_prefill_qkv(1, 2, 1, 256, 64, "cpu", seeds[0])
-        digest = float(qt.float().sum())
-        q.put((rank, t_max, units, rate, seeds, digest))
+        # this rank's shard: the same recipe drawn with its seed, through the oracle
+        o_sum, executed = _shard(seeds[0])
+        total_executed = bench.sum_over_ranks(float(executed))
+        q.put((rank, t_max, units, rate, seeds, o_sum, executed, total_executed))
     finally:
         dist.destroy_process_group()
+
+
+def _shard(seed):
+    """(sum of O, executed tiles) of the oracle on a small causal BLASST
+    prefill drawn with `seed` (B1, 2 query / 1 KV heads, 384 tokens, d 64,
+    tiles of 64, a = 10)."""
+    import math
+
+    import oracle
+    from block_sparse_attention_bsattn_b200 import inputs
+    N = 384
+    q, k, v = inputs.blasst_prefill_qkv(1, 2, 1, N, 64, "cpu", seed)
+    r = oracle.prefill(q, k, v, 64, 1 / math.sqrt(64), True, inputs.lambda_for(10, N))
+    return float(r["o"].sum()), int((r["status"] == 2).sum())
 
 
 def test_two_rank_reductions_and_seeds():
@@ -61,8 +77,13 @@ def test_two_rank_reductions_and_seeds():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    (r0, t0, u0, rate0, s0, d0), (r1, t1, u1, rate1, s1, d1) = res
+    (r0, t0, u0, rate0, s0, o0, e0, tot0), (r1, t1, u1, rate1, s1, o1, e1, tot1) = res
     assert t0 == t1 == 11.0                     # slowest rank
     assert u0 == u1 == 300.0                    # work of both ranks
     assert rate0 == rate1 == pytest.approx(300.0 / 11e-3)
-    assert s0 != s1 and d0 != d1                # different batches per rank
+    assert s0 != s1 and o0 != o1                # different batches per rank
+    # each rank's shard equals the same shard computed in one process, and
+    # the job's executed tiles are the sum of the shards'
+    (ro0, re0), (ro1, re1) = _shard(s0[0]), _shard(s1[0])
+    assert (o0, e0) == (ro0, re0) and (o1, e1) == (ro1, re1)
+    assert tot0 == tot1 == float(re0 + re1)
