@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include "bsattn.h"
+#include "backward_internal.h"
 #include "bsattn_internal.h"
 
 namespace bsattn {
@@ -357,6 +358,68 @@ int bsattn_fwd_decode_ex(const void* q, const void* k, const void* v, void* o, f
 
   CombineParams c{p.ws_o, p.ws_m, p.ws_l, static_cast<__nv_bfloat16*>(o), lse, num_splits, d};
   e = launch_decode_combine(c, B * Hq, d, stream);
+  return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}
+
+size_t bsattn_bwd_prefill_workspace_size(int B, int Hq, int N, int block) {
+  if (B < 1 || Hq < 1 || N < 1 || block < 1) return 0;
+  const size_t rows = (size_t)B * Hq * (size_t)((N + block - 1) / block) * 128;
+  return 2 * rows * sizeof(float);
+}
+
+int bsattn_bwd_prefill(const void* q, const void* k, const void* v, const void* o,
+                       const void* dout, const float* lse, const uint8_t* tile_status, void* dq,
+                       void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int block,
+                       float scale, int causal, const int32_t* d_seq_lens, void* workspace,
+                       size_t workspace_bytes, int32_t* d_status, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !tile_status || !dq || !dk || !dv || !workspace)
+    return BSATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || Hq % Hkv != 0) return BSATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return BSATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return BSATTN_ERR_UNSUPPORTED;
+  if (block != 128) return BSATTN_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, o, dout, dq, dk, dv, workspace};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return BSATTN_ERR_ALIGNMENT;
+  if (workspace_bytes < bsattn_bwd_prefill_workspace_size(B, Hq, N, block))
+    return BSATTN_ERR_CAPACITY;
+  const int64_t nq = (N + block - 1) / block;
+  if ((int64_t)B * Hq * nq > INT32_MAX || (int64_t)B * Hq * nq * 128 * 32 / 256 > INT32_MAX)
+    return BSATTN_ERR_UNSUPPORTED;
+  if (int rc = check_device()) return rc;
+
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_bf16_3d(&tq, q, d, N, (uint64_t)B * Hq, 128) ||
+      !encode_bf16_3d(&tk, k, d, N, (uint64_t)B * Hkv, 128) ||
+      !encode_bf16_3d(&tv, v, d, N, (uint64_t)B * Hkv, 128) ||
+      !encode_bf16_3d(&tdo, dout, d, N, (uint64_t)B * Hq, 128))
+    return BSATTN_ERR_CUDA;
+  const size_t rows = (size_t)B * Hq * (size_t)nq * 128;
+  BackwardParams p{};
+  p.o = static_cast<const __nv_bfloat16*>(o);
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.lse = lse;
+  p.tile_status = tile_status;
+  p.seq_lens = d_seq_lens;
+  p.ws_lse2 = static_cast<float*>(workspace);
+  p.ws_d = p.ws_lse2 + rows;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.status = d_status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.nq = (int)nq;
+  p.nk = (int)nq;
+  p.d = d;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  p.wait_limit_ns = g_wait_limit_ns;
+  const cudaError_t e = d == 128 ? launch_backward<128>(tq, tk, tv, tdo, p, stream)
+                                 : launch_backward<64>(tq, tk, tv, tdo, p, stream);
   return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
 

@@ -4,6 +4,7 @@
     python -m block_sparse_attention_bsattn_b200.microbench decode --batch 8 --a 10
     python -m block_sparse_attention_bsattn_b200.microbench videodit --heads 4
     python -m block_sparse_attention_bsattn_b200.microbench table4
+    python -m block_sparse_attention_bsattn_b200.microbench backward --heads 32 --a 10
 
 `table4` sweeps lambda = a / L on the B200 shapes of the BLASST page's Table 4
 (prefill: batch 148, 1 query / 1 KV head, 32K tokens, d 128, causal; decode:
@@ -115,10 +116,33 @@ def varlen(args):
     return rows
 
 
+def backward(args):
+    """Gradients of the causal BLASST prefill (B1, Hq heads, Hq/4 KV heads, N
+    tokens, d 128) with the forward's executed tiles held fixed.  Work per
+    executed tile: 5 GEMM tiles of 2*128*128*128 flops (S, dP, dV, dK, dQ);
+    the kernels issue 7 (S and dP again for dQ)."""
+    hkv = max(1, args.heads // 4)
+    q, k, v = inputs.blasst_prefill_qkv(1, args.heads, hkv, args.n, 128, "cuda", 1237)
+    lam = inputs.lambda_for(args.a, args.n)
+    nq = args.n // 128
+    st = torch.zeros(1, args.heads, nq, nq, dtype=torch.uint8, device="cuda")
+    o, lse = ops.bsattn_fwd_prefill(q, k, v, 128, None, True, lam, tile_status=st)
+    dout = torch.randn(q.shape, generator=torch.Generator(device="cuda").manual_seed(7),
+                       device="cuda").to(torch.bfloat16)
+    torch.cuda.synchronize()
+    exe = int((st == 2).sum())
+    fn = lambda: ops.bsattn_bwd_prefill(q, k, v, o, dout, lse, st, 128, None, True)  # noqa: E731
+    for _ in range(args.warmup):
+        fn()
+    ms = _time(fn, args.iters)
+    return {"heads": args.heads, "n": args.n, "a": args.a, "executed": exe, "ms": ms,
+            "tflops": 5 * TILE * exe / ms / 1e9, "tflops_issued": 7 * TILE * exe / ms / 1e9}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("what", choices=("prefill", "decode", "videodit", "mmdit", "table4",
-                                     "varlen"))
+                                     "varlen", "backward"))
     ap.add_argument("--heads", type=int, default=8, help="query heads (prefill/videodit/mmdit)")
     ap.add_argument("--n", type=int, default=32768, help="sequence length (prefill)")
     ap.add_argument("--batch", type=int, default=64, help="batch (decode)")
@@ -129,6 +153,10 @@ def main():
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--no-order", action="store_true", help="static masks: no longest-first order")
+    ap.add_argument("--dense-mask", action="store_true",
+                    help="videodit/mmdit: an all-ones mask of the same shape (same kernel)")
+    ap.add_argument("--diag-mask", action="store_true",
+                    help="videodit/mmdit: only the diagonal block of every row")
     ap.add_argument("--reverse", action="store_true", help="prefill: descending visit order")
     ap.add_argument("--skip-v", action="store_true", help="prefill: load V only for kept tiles")
     ap.add_argument("--sink-seed", action="store_true", help="decode: sink-seeded splits")
@@ -142,6 +170,10 @@ def main():
         nq = args.n // 128
         st = torch.zeros(1, args.heads, nq, nq, dtype=torch.uint8, device="cuda")
         opt = dict(reverse=args.reverse, skip_v=args.skip_v)
+        if args.diag_mask:   # one key tile per query tile: the per-work-item cost
+            m = torch.eye(nq, dtype=torch.uint8)[None].cuda()
+            rp, ci, _ = ops.bsattn_build_index(m, 128, 128, True)
+            opt.update(row_ptr=rp, col_idx=ci, mask_heads=1)
         o, _ = ops.bsattn_fwd_prefill(q, k, v, 128, None, True, lam, tile_status=st, **opt)
         torch.cuda.synchronize()
         vis, exe = int((st > 0).sum()), int((st == 2).sum())
@@ -156,7 +188,12 @@ def main():
     elif args.what in ("videodit", "mmdit"):
         w = inputs.workload(args.what, device="cuda", generate=False)
         q, k, v = inputs.normal_qkv(1, args.heads, args.heads, w.N, w.d, "cuda", 1236)
-        m = w.mask.cuda()
+        if args.dense_mask:
+            m = torch.ones_like(w.mask).cuda()
+        elif args.diag_mask:   # one key tile per query tile: the per-work-item cost
+            m = torch.eye(w.nq, dtype=torch.uint8)[None].cuda()
+        else:
+            m = w.mask.cuda()
         rp, ci, nnz, order = ops.bsattn_build_index(m, w.block, w.block, False, with_order=True)
         if args.no_order:
             order = None
@@ -167,11 +204,14 @@ def main():
         ms = _time(fn, args.iters)
         tiles = int(nnz.sum()) * args.heads
         flops = 4 * w.block * w.block * w.d * tiles
-        out.update(heads=args.heads, n=w.N, d=w.d, tiles=tiles, ms=ms, tflops=flops / ms / 1e9)
+        out.update(heads=args.heads, n=w.N, d=w.d, tiles=tiles, dense_mask=args.dense_mask, ms=ms,
+                   tflops=flops / ms / 1e9)
     elif args.what == "table4":
         out["rows"] = table4(args)
     elif args.what == "varlen":
         out["rows"] = varlen(args)
+    elif args.what == "backward":
+        out.update(backward(args))
     else:
         B, Hq, Hkv, L, d = args.batch, 32, args.hkv, args.l, 128
         ns = args.splits

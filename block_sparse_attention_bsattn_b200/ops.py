@@ -59,6 +59,11 @@ _lib.bsattn_fwd_decode_ex.restype = _I
 _lib.bsattn_fwd_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I,
                                            _F, _I, _P, _P, _P]
 _lib.bsattn_fwd_decode_noalloc.restype = _I
+_lib.bsattn_bwd_prefill_workspace_size.argtypes = [_I, _I, _I, _I]
+_lib.bsattn_bwd_prefill_workspace_size.restype = _SZ
+_lib.bsattn_bwd_prefill.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
+                                    _I, _F, _I, _P, _P, _SZ, _P, _P]
+_lib.bsattn_bwd_prefill.restype = _I
 
 # option bits of the _ex entry points (include/bsattn.h)
 PREFILL_REVERSE = 0x1
@@ -70,7 +75,8 @@ EXPORTED = ("bsattn_status_string", "bsattn_version", "bsattn_debug_set", "bsatt
             "bsattn_fwd_prefill", "bsattn_fwd_prefill_ex", "bsattn_fwd_prefill_host",
             "bsattn_decode_workspace_size",
             "bsattn_fwd_decode", "bsattn_fwd_decode_ex",
-            "bsattn_fwd_decode_noalloc")
+            "bsattn_fwd_decode_noalloc", "bsattn_bwd_prefill_workspace_size",
+            "bsattn_bwd_prefill")
 
 
 class BsattnError(RuntimeError):
@@ -334,5 +340,41 @@ def bsattn_fwd_decode_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                         int(num_splits), _ptr(tile_status), _ptr(status),
                                         _stream(stream))
     if rc:
-        raise BsattnError(rc, "bsattn_fwd_decode_noalloc")
+        raise BsattnError(rc, "bsattn_fwd_decode_noalloc", "bsattn_bwd_prefill_workspace_size",
+            "bsattn_bwd_prefill")
     return o, lse
+
+
+def bsattn_bwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                       dout: torch.Tensor, lse: torch.Tensor, tile_status: torch.Tensor,
+                       block: int = 128, scale: Optional[float] = None, causal: bool = False,
+                       seq_lens: Optional[torch.Tensor] = None,
+                       status: Optional[torch.Tensor] = None, stream=None):
+    """Gradients of bsattn_fwd_prefill with its executed tiles held fixed:
+    (dq [B,Hq,N,d], dk, dv [B,Hkv,N,d]) bf16.  lse and tile_status are the
+    forward call's outputs; only tiles marked 2 (executed) take part."""
+    for t, name in ((q, "q"), (o, "o"), (dout, "dout"), (k, "k"), (v, "v")):
+        _check(t, name, torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    _check(tile_status, "tile_status", torch.uint8, 4)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    nq = -(-N // block)
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape or o.shape != q.shape or \
+            dout.shape != q.shape or lse.shape != (B, Hq, N) or \
+            tile_status.shape != (B, Hq, nq, nq):
+        raise ValueError("shapes do not match the forward call's")
+    if seq_lens is not None:
+        _check(seq_lens, "seq_lens", torch.int32, 1)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    ws_bytes = int(_lib.bsattn_bwd_prefill_workspace_size(B, Hq, N, int(block)))
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rc = _lib.bsattn_bwd_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                 _ptr(tile_status), _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, N,
+                                 d, int(block), float(scale), int(causal), _ptr(seq_lens),
+                                 _ptr(ws), ws_bytes, _ptr(status), _stream(stream))
+    if rc:
+        raise BsattnError(rc, "bsattn_bwd_prefill")
+    return dq, dk, dv

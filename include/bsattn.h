@@ -328,6 +328,46 @@ int bsattn_fwd_decode_noalloc(const void *q, const void *k, const void *v, void 
                               int causal, float lambda, int num_splits, uint8_t *tile_status,
                               int32_t *d_status, cudaStream_t stream);
 
+/*
+ * bsattn_bwd_prefill_workspace_size -- bytes of scratch bsattn_bwd_prefill
+ * needs: two fp32 values (D and LSE in base 2) per query row, padded to
+ * whole query tiles.
+ */
+size_t bsattn_bwd_prefill_workspace_size(int B, int Hq, int N, int block);
+
+/*
+ * bsattn_bwd_prefill -- gradients of bsattn_fwd_prefill for sparsity-aware
+ * training ("BLASST: Dynamic Blocked Attention Sparsity via Softmax
+ * Thresholding", section 3.3: fine-tuning runs the forward with the skip, and
+ * the blocks it skipped receive no gradient because they were never
+ * computed).  With the forward's executed tiles held fixed, the forward is the
+ * softmax attention over their keys, and this is its exact gradient:
+ *   P = exp(scale Q K^T - LSE), D = rowsum(dO * O), dS = P (dO V^T - D),
+ *   dV = P^T dO, dK = scale dS^T Q, dQ = scale dS K,
+ * summed over the executed tiles only; keys in tiles that no query tile
+ * executed get dK = dV = 0.
+ *
+ *   q, k, v, o      the forward's inputs and output (bf16, layouts as there)
+ *   dout            dL/dO, bf16 [B][Hq][N][d]
+ *   lse             the forward's LSE, fp32 [B][Hq][N] (required)
+ *   tile_status     the forward's tile status, uint8 [B][Hq][nq][nk]
+ *                   (required; only tiles marked 2, executed, take part)
+ *   dq              bf16 [B][Hq][N][d];  dk, dv bf16 [B][Hkv][N][d] (written)
+ *   causal, d_seq_lens  as in the forward call
+ *   workspace       device scratch of bsattn_bwd_prefill_workspace_size bytes,
+ *                   16-byte aligned, owned by the caller
+ *
+ * block must be 128 and d 64 or 128 (else BSATTN_ERR_UNSUPPORTED).  Three
+ * kernels run on `stream`: per-row statistics, then dK/dV (one CTA per key
+ * tile, accumulating over the GQA group's query heads) and dQ (one CTA per
+ * query tile); each output tile has a single writer, no atomics.
+ */
+int bsattn_bwd_prefill(const void *q, const void *k, const void *v, const void *o,
+                       const void *dout, const float *lse, const uint8_t *tile_status, void *dq,
+                       void *dk, void *dv, int B, int Hq, int Hkv, int N, int d, int block,
+                       float scale, int causal, const int32_t *d_seq_lens, void *workspace,
+                       size_t workspace_bytes, int32_t *d_status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

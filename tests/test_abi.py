@@ -165,3 +165,25 @@ def test_shipped_library_has_no_trace_buffer(lib):
     assert not view
     assert lib.bsattn_debug_trace(0, None) == 0
     assert lib.bsattn_debug_trace(-1, None) == -1
+
+
+def test_backward_host_validation(lib):
+    """bsattn_bwd_prefill rejects bad arguments before touching a device."""
+    f = lib.bsattn_bwd_prefill
+    assert lib.bsattn_bwd_prefill_workspace_size(1, 2, 300, 128) == 2 * (2 * 3 * 128) * 4
+
+    def call(q=0x1000, st=0x9000, d=128, block=128, hq=4, hkv=2, scale=0.1, ws=0xa000,
+             wsb=1 << 20, dq=0xb000):
+        return f(P(q) if q else None, P(0x2000), P(0x3000), P(0x4000), P(0x5000), P(0x6000),
+                 P(st) if st else None, P(dq), P(0xc000), P(0xd000), 1, hq, hkv, 300, d, block,
+                 ctypes.c_float(scale), 1, None, P(ws) if ws else None, wsb, None, None)
+    assert call(q=0) == -1
+    assert call(st=0) == -1             # the forward's tile status is required
+    assert call(ws=0) == -1
+    assert call(hq=3, hkv=2) == -1
+    assert call(scale=0.0) == -1
+    assert call(d=96) == -2
+    assert call(block=64) == -2         # 128-token tiles only
+    assert call(q=0x1008) == -3
+    assert call(dq=0xb004) == -3
+    assert call(wsb=100) == -4          # workspace too small
