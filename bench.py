@@ -391,12 +391,9 @@ def time_calls(fn, n, flush=None):
 
 
 def static_kernel_name(w):
-    """The kernel bsattn_fwd_prefill dispatches a one-mask, one-query-head-per-KV-head
-    workload to: 64-token tiles run one query tile per CTA, 128-token tiles two
-    query tiles with visit lists of their own."""
-    if w.block == 64:
-        return f"prefill_kernel<{w.d}, 64, 0>"
-    return f"prefill_duo_kernel<{w.d}, 0>"
+    """The kernel bsattn_fwd_prefill dispatches a block mask with one query
+    head per KV head to: one query tile per CTA."""
+    return f"prefill_kernel<{w.d}, {w.block}, 0>"
 
 
 def static_section(iters, warmup, peak):
@@ -516,6 +513,37 @@ def oracle_per_config(pw, dw, a):
     return out
 
 
+def backward_section(step, iters, warmup, peak):
+    """Gradients of the step's BLASST prefill (same inputs, same a) with its
+    executed tiles held fixed (bsattn_bwd_prefill: a row kernel, dK/dV, dQ).
+    Work: 5 GEMM tiles of 2*128^3 flops per executed tile (S, dP, dV, dK, dQ;
+    the kernels issue 7, recomputing S and dP for dQ)."""
+    from block_sparse_attention_bsattn_b200 import ops
+    pw = step.pw
+    st = torch.zeros(pw.B, pw.Hq, pw.nq, pw.nk, dtype=torch.uint8, device="cuda")
+    step.index()
+    step.prefill(st)
+    g = torch.Generator(device="cuda").manual_seed(4242)
+    dout = torch.randn(pw.q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(pw.q), torch.empty_like(pw.k), torch.empty_like(pw.v)
+    ws = torch.empty(ops.bsattn_bwd_prefill_workspace_size(pw.B, pw.Hq, pw.N, BLK),
+                     dtype=torch.uint8, device="cuda")
+    fn = lambda: ops.bsattn_bwd_prefill(pw.q, pw.k, pw.v, step.o, dout, step.lse, st, BLK,  # noqa: E731
+                                        pw.scale, True, status=step.status, dq=dq, dk=dk, dv=dv,
+                                        workspace=ws)
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(time_calls(fn, iters))
+    exe = int((st == 2).sum())
+    flops = 5 * TILE_FLOP * exe
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"kernels": "bwd_rows_kernel + bwd_dkdv_kernel<128> + bwd_dq_kernel<128>",
+            "ms": ms, "tflops": tf, "frac": tf / peak, "flops_per_call": flops,
+            "issued_tflops": 7 * TILE_FLOP * exe / (ms * 1e-3) / 1e12,
+            "executed_tiles": exe, "a": step.a}
+
+
 # ------------------------------------------------------------------ main
 def config_dict(pw, dw, a, n):
     return {
@@ -584,6 +612,7 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-static", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -702,6 +731,11 @@ def main():
                           "d2h_bytes_per_step": byts[3],
                           "note": "KV cache resident on the device; the query and O cross PCIe"}}
 
+    bwd = None
+    if not args.no_backward:
+        bwd = backward_section(step, max(3, K // 4), 2, peaks["bf16_tflops"])
+        assert step.status.item() == 0
+
     static = None
     if not args.no_static:
         clocks_s = ClockSampler(local)
@@ -773,6 +807,7 @@ def main():
         "sweep": sweep,
         "variants": variants,
         "static": static,
+        "backward": bwd,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": Step.LAUNCHES * K,

@@ -1,6 +1,7 @@
 // Host side of the C ABI declared in include/bsattn.h: argument validation,
 // TMA tensor-map encoding (through the driver entry point, so the library
 // needs no link-time libcuda), kernel attribute set-up and launches.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -241,15 +242,13 @@ int bsattn_fwd_prefill_ex(const void* q, const void* k, const void* v, void* o, 
                  : launch_prefill_pair<64>(tq, tk, tv, p, (int)pitems, stream);
     return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
   }
-  // Block masks whose rows no two query tiles share (one query head per KV
-  // head with a mask, or one mask per head): two query tiles per CTA with
-  // visit lists of their own, streamed through one ring.  V skipping keeps
-  // the one-tile kernel, which has a warp for conditional V loads.
-  if (block == 128 && !p.skip_v) {
-    const int64_t dgrid = (items + 1) / 2;
-    e = d == 128 ? launch_prefill_duo<128>(tq, tk, tv, p, (int)dgrid, stream)
-                 : launch_prefill_duo<64>(tq, tk, tv, p, (int)dgrid, stream);
-    return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+  // one query tile per CTA: the longest rows of every head first (about one
+  // wave of them), then head by head
+  {
+    const int sms = sm_count();
+    if (sms <= 0) return BSATTN_ERR_CUDA;
+    const int64_t bh = (int64_t)B * Hq;
+    p.lead_ranks = (int)std::min<int64_t>(nq, (sms + bh - 1) / bh);
   }
   if (d == 128 && block == 128) e = launch_prefill<128, 128>(tq, tk, tv, p, (int)items, stream);
   else if (d == 64 && block == 128) e = launch_prefill<64, 128>(tq, tk, tv, p, (int)items, stream);

@@ -34,6 +34,7 @@ struct PrefillParams {
   int use_skip;      // lambda > 0
   int debug_stall;   // test hook: the query tile is withheld from the tensor core
   int pair_tiles;    // two-slot kernel: consecutive query tiles of one head
+  int lead_ranks;    // one-tile kernel: rows of rank < lead_ranks of every head go first
   int reverse;       // visit each row's key tiles in descending order
   int skip_v;        // load V only for tiles some query tile keeps
   const int32_t* seq_lens;   // [B] valid tokens per sequence (key padding) or null
@@ -79,11 +80,6 @@ template <int D>
 cudaError_t launch_prefill_pair(const CUtensorMap& tq, const CUtensorMap& tk,
                                 const CUtensorMap& tv, const PrefillParams& p, int grid,
                                 cudaStream_t stream);
-
-template <int D>
-cudaError_t launch_prefill_duo(const CUtensorMap& tq, const CUtensorMap& tk,
-                               const CUtensorMap& tv, const PrefillParams& p, int grid,
-                               cudaStream_t stream);
 
 template <int D, int BLK, int G>
 cudaError_t launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv,

@@ -106,21 +106,35 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // ---- work item: head by head (the heads of one KV head are adjacent, so
-  // the CTAs resident at one time share a K/V stream that stays in L2).
-  // Inside a head, a row order from the index builder (longest rows first),
-  // else causal work longest first, else ascending query tiles.
-  int i, bh;
+  // ---- work item.  Query tiles are ranked inside each head: by the index
+  // builder's row order (longest rows first), else causal work longest first,
+  // else ascending.  The lead_ranks best-ranked (longest) rows of every head
+  // go first, all heads at once, so that no head's longest rows start late
+  // and run on alone at the end of the launch; the rest go head by head (the
+  // heads of one KV head are adjacent, so the CTAs resident at one time share
+  // a K/V stream that stays in L2).
+  int rank, bh;
+  {
+    const int BH = p.B * p.Hq;
+    const int lead = p.lead_ranks;
+    const int64_t x = blockIdx.x;
+    if (x < (int64_t)lead * BH) {
+      rank = (int)(x / BH);
+      bh = (int)(x - (int64_t)rank * BH);
+    } else {
+      const int64_t y = x - (int64_t)lead * BH;
+      bh = (int)(y / (p.nq - lead));
+      rank = lead + (int)(y - (int64_t)bh * (p.nq - lead));
+    }
+  }
+  int i;
   if (p.row_order) {
-    bh = (int)(blockIdx.x / p.nq);
     const int mh_o = p.mask_heads == 1 ? 0 : bh % p.Hq;
-    i = p.row_order[(int64_t)mh_o * p.nq + (int)(blockIdx.x % p.nq)];
+    i = p.row_order[(int64_t)mh_o * p.nq + rank];
   } else if (p.causal) {
-    bh = (int)(blockIdx.x / p.nq);
-    i = p.nq - 1 - (int)(blockIdx.x % p.nq);
+    i = p.nq - 1 - rank;
   } else {
-    bh = (int)(blockIdx.x / p.nq);
-    i = (int)(blockIdx.x % p.nq);
+    i = rank;
   }
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int kvh = h / (p.Hq / p.Hkv);

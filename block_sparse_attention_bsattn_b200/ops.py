@@ -345,14 +345,22 @@ def bsattn_fwd_decode_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return o, lse
 
 
+def bsattn_bwd_prefill_workspace_size(B: int, Hq: int, N: int, block: int = 128) -> int:
+    return int(_lib.bsattn_bwd_prefill_workspace_size(B, Hq, N, int(block)))
+
+
 def bsattn_bwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
                        dout: torch.Tensor, lse: torch.Tensor, tile_status: torch.Tensor,
                        block: int = 128, scale: Optional[float] = None, causal: bool = False,
                        seq_lens: Optional[torch.Tensor] = None,
-                       status: Optional[torch.Tensor] = None, stream=None):
+                       status: Optional[torch.Tensor] = None, stream=None,
+                       dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+                       dv: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None):
     """Gradients of bsattn_fwd_prefill with its executed tiles held fixed:
     (dq [B,Hq,N,d], dk, dv [B,Hkv,N,d]) bf16.  lse and tile_status are the
-    forward call's outputs; only tiles marked 2 (executed) take part."""
+    forward call's outputs; only tiles marked 2 (executed) take part.  dq, dk,
+    dv and the workspace may be passed in (else they are allocated here)."""
     for t, name in ((q, "q"), (o, "o"), (dout, "dout"), (k, "k"), (v, "v")):
         _check(t, name, torch.bfloat16, 4)
     _check(lse, "lse", torch.float32, 3)
@@ -369,8 +377,21 @@ def bsattn_bwd_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     ws_bytes = int(_lib.bsattn_bwd_prefill_workspace_size(B, Hq, N, int(block)))
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    else:
+        if not workspace.is_cuda or not workspace.is_contiguous() or \
+                workspace.numel() * workspace.element_size() < ws_bytes:
+            raise ValueError(f"workspace: a contiguous CUDA buffer of {ws_bytes} bytes needed")
+        ws = workspace
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check_buf(dq, "dq", torch.bfloat16, q.numel(), exact=True)
+    _check_buf(dk, "dk", torch.bfloat16, k.numel(), exact=True)
+    _check_buf(dv, "dv", torch.bfloat16, v.numel(), exact=True)
+    _check_buf(status, "status", torch.int32, 1)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
     rc = _lib.bsattn_bwd_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
                                  _ptr(tile_status), _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, N,
                                  d, int(block), float(scale), int(causal), _ptr(seq_lens),

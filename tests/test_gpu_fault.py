@@ -22,10 +22,10 @@ def _ops():
 
 
 # two heads of one KV head (pair kernel, heads mode), one head (pair kernel,
-# two consecutive query tiles), 64-token tiles (one-query-tile kernel), a
-# block mask with one query head per KV head (two query tiles with visit
-# lists of their own); lambda > 0 runs the variants with the skip vote, whose
-# warps must all still meet at the vote barrier after the wait ran out
+# two consecutive query tiles), 64-token tiles and a block mask with one
+# query head per KV head (one-query-tile kernel); lambda > 0 runs the
+# variants with the skip vote, whose warps must all still meet at the vote
+# barrier after the wait ran out
 @pytest.mark.parametrize("hq,hkv,block,masked", [(2, 1, 128, False), (1, 1, 128, False),
                                                  (1, 1, 64, False), (2, 2, 128, True)])
 @pytest.mark.parametrize("lam", [0.0, 1e-3])

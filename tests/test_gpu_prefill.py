@@ -374,11 +374,10 @@ def test_blasst_prefill_full_size_sampled(a):
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("lam", [0.0, 3e-3])
 @pytest.mark.parametrize("per_head", [False, True])
-def test_two_tile_kernel_own_lists(d, causal, lam, per_head):
+def test_masks_rows_of_their_own(d, causal, lam, per_head):
     """Masks whose rows no two query tiles share (one query head per KV head,
-    or one mask per head) run two query tiles per CTA, each with its own
-    visit list: an odd number of query tiles (the last CTA holds one), rows
-    of very different lengths, empty rows and a ragged tail."""
+    or one mask per head) with 128-token tiles: an odd number of query tiles,
+    rows of very different lengths, empty rows and a ragged tail."""
     rng = np.random.default_rng(d + 2 * causal + (lam > 0) + 4 * per_head)
     B, Hq, Hkv, N = 1, 3, 3 if not per_head else 1, 5 * 128 - 17
     nb = -(-N // 128)
