@@ -762,10 +762,11 @@ def main():
 
     bf16_peak = peaks["bf16_tflops"]
     hbm_peak = peaks["hbm_gbs"]
-    prefill_roof = {"kernel": "prefill_pair_kernel<128, 0> (two GQA heads per CTA)",
+    prefill_roof = {"kernel": "prefill_pair_kernel<128, 0, %d> (two GQA heads per CTA%s)"
+                              % (int(args.a > 0), ", skip vote" if args.a > 0 else ""),
                     "bound": "tensor", "achieved": tf_rank, "peak": bf16_peak,
                     "unit": "TFLOP/s", "frac": tf_rank / bf16_peak,
-                    "traffic": profiled_traffic("prefill_pair_kernel<128, 0>"),
+                    "traffic": profiled_traffic("prefill_pair_kernel<128, 0, %d>" % int(args.a > 0)),
                     "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
                     "flops_per_launch": p_flops,
                     "strict_flops_per_launch": strict_flops,
