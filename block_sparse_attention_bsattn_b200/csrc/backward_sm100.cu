@@ -24,8 +24,10 @@
 //                    S, dQ += dS K accumulated in TMEM; one bf16 write of dQ.
 // No atomics: each output tile has one writer.  Warps: 0 TMA producer (it also
 // finds the executed tiles, 32 status bytes per ballot, and passes each one to
-// the other roles through its stage), 1 MMA issuer, 4..7 the element-wise
-// work, one thread per TMEM lane.  Every wait is bounded in time.
+// the other roles through its stage), 1 MMA issuer, 4..11 the element-wise
+// work: two warps per TMEM lane quarter, each owning half of the tile's
+// columns and writing its bf16 results inside them.  Every wait is bounded
+// in time.
 #include <cmath>
 #include <cstdint>
 #include <cuda.h>
@@ -101,7 +103,7 @@ struct BwdCfg {
   static constexpr uint32_t ACC1 = D;               // dV (dK/dV kernel)
   static constexpr uint32_t S_COL = 256;            // S or S^T, then P^T / dS in bf16
   static constexpr uint32_t DP_COL = 384;           // dP or dP^T, then dS^T in bf16
-  static constexpr int THREADS = 256;
+  static constexpr int THREADS = 384;              // 4 role warps + 8 element-wise warps
 };
 
 struct BwdBarriers {
@@ -116,6 +118,14 @@ struct BwdBarriers {
   int meta[2][2];              // per stage: (head, query tile) / (key tile, -) or -1 = end
 };
 
+// TMEM column (relative to S or dP) of the bf16 pairs of K-step kk (16 of
+// the 128 inner indices) of the element-wise results: the warps that own
+// inner indices [64 h, 64 h + 64) write their 32 columns of pairs at 64 h,
+// inside the 64 fp32 columns they alone read.
+__device__ __forceinline__ uint32_t bf16_col(int kk) {
+  return (uint32_t)((kk / 4) * 64 + (kk % 4) * 8);
+}
+
 // Producer's end-of-stream marker in stage t % 2 (no bytes: a plain arrive).
 __device__ __forceinline__ bool bwd_end_marker(BwdBarriers* bars, int t, volatile int* abort,
                                                uint64_t lim) {
@@ -128,7 +138,7 @@ __device__ __forceinline__ bool bwd_end_marker(BwdBarriers* bars, int t, volatil
 
 // ------------------------------------------------------------------ dK, dV
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const BackwardParams p) {
@@ -155,7 +165,7 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(&bars->st_empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->p_ready, 4);
+    mbar_init(&bars->p_ready, 8);
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -269,12 +279,12 @@ __global__ void __launch_bounds__(256, 1)
         // B = the query-side tile read MN-major
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tmem + C::ACC1, tmem + C::S_COL + kk * 8,
+          mma_ts(tmem + C::ACC1, tmem + C::S_COL + bf16_col(kk),
                  smem_desc(da + kk * (16 * 128), C::T_HALF, 1024, 2), IDESC_O,
                  (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tmem + C::ACC0, tmem + C::DP_COL + kk * 8,
+          mma_ts(tmem + C::ACC0, tmem + C::DP_COL + bf16_col(kk),
                  smem_desc(qa + kk * (16 * 128), C::T_HALF, 1024, 2), IDESC_O,
                  (t > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->st_empty[st]);
@@ -285,11 +295,16 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp >= 4) {
     // ======================================================== element-wise warps
+    // Two warps per TMEM lane quarter: warp half hc owns the query columns
+    // [64 hc, 64 hc + 64) of its 32 key rows and writes their bf16 pairs at
+    // column 64 hc, inside the columns only it reads.
     const int quarter = warp % 4;
+    const int hc = (warp - 4) / 4;
     const int c = quarter * 32 + lane;           // key row of the tile
     const int key = j * 128 + c;
     const bool key_ok = key < len;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
     int t = 0;
     bool ok = true;
     for (;; ++t) {
@@ -309,37 +324,51 @@ __global__ void __launch_bounds__(256, 1)
           reinterpret_cast<const float*>(smem + C::KV_STG + st * C::KV_STG_BYTES + 2 * C::T_BYTES);
       const float* dvec = lse2 + 128;
       const int q0 = ii * 128;
-      // 32 query columns at a time; the bf16 results go to columns already read
+      // a query tile after the key tile sees every key (causal), so only the
+      // diagonal pair needs the per-element mask
+      const bool diag = p.causal && ii == j;
 #pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c0 = 64 * hc + 32 * cc;        // 32 query columns
         uint32_t s[32], dp[32];
         tmem_ld32(lane_addr + C::S_COL + c0, s);
         tmem_ld32(lane_addr + C::DP_COL + c0, dp);
         tmem_wait_ld();
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int r = 0; r < 32; r += 2) {
-          float pv[2], ds[2];
+        for (int r = 0; r < 32; r += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + r);
+          const float4 d4 = *reinterpret_cast<const float4*>(dvec + c0 + r);
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int qr = c0 + r + u;
-            const bool on = key_ok && (!p.causal || key <= q0 + qr);
-            const float x = __uint_as_float(s[r + u]) * p.scale_log2 - lse2[qr];
-            pv[u] = on ? fast_exp2(x) : 0.f;
-            ds[u] = pv[u] * (__uint_as_float(dp[r + u]) - dvec[qr]) * p.scale;
+          for (int u = 0; u < 4; u += 2) {
+            const float2 lu = u == 0 ? make_float2(-l4.x, -l4.y) : make_float2(-l4.z, -l4.w);
+            const float2 du = u == 0 ? make_float2(-d4.x, -d4.y) : make_float2(-d4.z, -d4.w);
+            const float2 x = ffma2(make_float2(__uint_as_float(s[r + u]),
+                                               __uint_as_float(s[r + u + 1])), sl2, lu);
+            float2 pv = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            if (!key_ok) pv = make_float2(0.f, 0.f);
+            if (diag) {
+              if (key > q0 + c0 + r + u) pv.x = 0.f;
+              if (key > q0 + c0 + r + u + 1) pv.y = 0.f;
+            }
+            const float2 g = fadd2(make_float2(__uint_as_float(dp[r + u]),
+                                               __uint_as_float(dp[r + u + 1])), du);
+            const float2 ds = ffma2(make_float2(pv.x * p.scale, pv.y * p.scale), g,
+                                    make_float2(0.f, 0.f));
+            pk[(r + u) / 2] = pack_bf16x2(pv.x, pv.y);
+            dk[(r + u) / 2] = pack_bf16x2(ds.x, ds.y);
           }
-          pk[r / 2] = pack_bf16x2(pv[0], pv[1]);
-          dk[r / 2] = pack_bf16x2(ds[0], ds[1]);
         }
-        tmem_st16(lane_addr + C::S_COL + c0 / 2, pk);
-        tmem_st16(lane_addr + C::DP_COL + c0 / 2, dk);
+        tmem_st16(lane_addr + C::S_COL + 64 * hc + 16 * cc, pk);
+        tmem_st16(lane_addr + C::DP_COL + 64 * hc + 16 * cc, dk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready);
     }
-    // ---- epilogue: dK and dV rows of this key tile (zero when no pair)
+    // ---- epilogue: the key tile's dK rows (warp half 0) and dV rows (half 1),
+    // zero when no pair took part
     if (ok) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->acc_done, 0, abort, lim))) ok = false;
       tc_fence_after();
@@ -347,27 +376,24 @@ __global__ void __launch_bounds__(256, 1)
     if (ok) {
       const bool in_buf = key < p.N;
       const int64_t row = ((int64_t)(b * p.Hkv + kvh) * p.N + key) * D;
+      __nv_bfloat16* dst = (hc == 0 ? p.dk : p.dv) + row;
+      const uint32_t col = hc == 0 ? C::ACC0 : C::ACC1;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16* dst = (which == 0 ? p.dk : p.dv) + row;
-        const uint32_t col = which == 0 ? C::ACC0 : C::ACC1;
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
+        if (t > 0) {
+          tmem_ld32(lane_addr + col + c0, r);
+          tmem_wait_ld();
+        }
+        if (in_buf) {
+          uint32_t w[16];
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t r[32];
-          if (t > 0) {
-            tmem_ld32(lane_addr + col + c0, r);
-            tmem_wait_ld();
-          }
-          if (in_buf) {
-            uint32_t w[16];
+          for (int x = 0; x < 32; x += 2)
+            w[x / 2] = t > 0 ? pack_bf16x2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])) : 0u;
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll
-            for (int x = 0; x < 32; x += 2)
-              w[x / 2] = t > 0 ? pack_bf16x2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])) : 0u;
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-          }
+          for (int v = 0; v < 4; ++v)
+            d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
     }
@@ -384,7 +410,7 @@ __global__ void __launch_bounds__(256, 1)
 
 // ------------------------------------------------------------------ dQ
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const BackwardParams p) {
@@ -412,7 +438,7 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(&bars->st_empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->p_ready, 4);
+    mbar_init(&bars->p_ready, 8);
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -518,7 +544,7 @@ __global__ void __launch_bounds__(256, 1)
         // dQ += dS K (scale folded into dS): A from TMEM, B = the K tile read MN-major
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tmem + C::ACC0, tmem + C::S_COL + kk * 8,
+          mma_ts(tmem + C::ACC0, tmem + C::S_COL + bf16_col(kk),
                  smem_desc(ka + kk * (16 * 128), C::T_HALF, 1024, 2), IDESC_O,
                  (t > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->st_empty[st]);
@@ -529,13 +555,20 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp >= 4) {
     // ======================================================== element-wise warps
+    // Two warps per TMEM lane quarter: warp half hc owns the key columns
+    // [64 hc, 64 hc + 64) of its 32 query rows and writes their bf16 pairs at
+    // column 64 hc, inside the columns only it reads.
     const int quarter = warp % 4;
+    const int hc = (warp - 4) / 4;
     const int rr = quarter * 32 + lane;          // query row of the tile
     const int qpos = i * 128 + rr;
     const int64_t wrow = ((int64_t)(b * p.Hq + h) * p.nq + i) * 128 + rr;
     const float lse2 = p.ws_lse2[wrow];          // +inf for rows without weight
     const float dval = p.ws_d[wrow];
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+    const float2 nl2 = make_float2(-lse2, -lse2);
+    const float2 nd2 = make_float2(-dval, -dval);
     int t = 0;
     bool ok = true;
     for (;; ++t) {
@@ -552,8 +585,12 @@ __global__ void __launch_bounds__(256, 1)
       }
       tc_fence_after();
       const int k0 = j * 128;
+      // a key tile before the query tile and inside the sequence needs no
+      // per-element mask
+      const bool masked = (p.causal && j == i) || k0 + 128 > len;
 #pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c0 = 64 * hc + 32 * cc;        // 32 key columns
         uint32_t s[32], dp[32];
         tmem_ld32(lane_addr + C::S_COL + c0, s);
         tmem_ld32(lane_addr + C::DP_COL + c0, dp);
@@ -561,24 +598,29 @@ __global__ void __launch_bounds__(256, 1)
         uint32_t dk[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
-          float ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int key = k0 + c0 + x + u;
-            const bool on = key < len && (!p.causal || key <= qpos);
-            const float pv = on ? fast_exp2(__uint_as_float(s[x + u]) * p.scale_log2 - lse2) : 0.f;
-            ds[u] = pv * (__uint_as_float(dp[x + u]) - dval) * p.scale;
+          const float2 y = ffma2(make_float2(__uint_as_float(s[x]), __uint_as_float(s[x + 1])),
+                                 sl2, nl2);
+          float2 pv = make_float2(fast_exp2(y.x), fast_exp2(y.y));
+          if (masked) {
+            const int key = k0 + c0 + x;
+            if (key >= len || (p.causal && key > qpos)) pv.x = 0.f;
+            if (key + 1 >= len || (p.causal && key + 1 > qpos)) pv.y = 0.f;
           }
-          dk[x / 2] = pack_bf16x2(ds[0], ds[1]);
+          const float2 g = fadd2(make_float2(__uint_as_float(dp[x]), __uint_as_float(dp[x + 1])),
+                                 nd2);
+          const float2 ds = ffma2(make_float2(pv.x * p.scale, pv.y * p.scale), g,
+                                  make_float2(0.f, 0.f));
+          dk[x / 2] = pack_bf16x2(ds.x, ds.y);
         }
-        tmem_st16(lane_addr + C::S_COL + c0 / 2, dk);
+        tmem_st16(lane_addr + C::S_COL + 64 * hc + 16 * cc, dk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready);
     }
-    // ---- epilogue: this query tile's dQ rows (zero when no key tile)
+    // ---- epilogue: this query tile's dQ rows, columns [hc D/2, hc D/2 + D/2)
+    // per warp half (zero when no key tile took part)
     if (ok) {
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->acc_done, 0, abort, lim))) ok = false;
       tc_fence_after();
@@ -587,7 +629,7 @@ __global__ void __launch_bounds__(256, 1)
       const bool in_buf = qpos < p.N;
       __nv_bfloat16* dst = p.dq + ((int64_t)(b * p.Hq + h) * p.N + qpos) * D;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = hc * (D / 2); c0 < hc * (D / 2) + D / 2; c0 += 32) {
         uint32_t rg[32];
         if (t > 0) {
           tmem_ld32(lane_addr + C::ACC0 + c0, rg);
