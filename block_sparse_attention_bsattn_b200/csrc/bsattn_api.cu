@@ -108,6 +108,11 @@ int bsattn_debug_set(long long wait_limit_ns, int inject_stall) {
   return BSATTN_OK;
 }
 
+int bsattn_debug_exp2(const float* d_x, float* d_y, int64_t n, cudaStream_t stream) {
+  if (n < 0 || n > ((int64_t)1 << 32) || (n > 0 && (!d_x || !d_y))) return BSATTN_ERR_INVALID_ARG;
+  return launch_exp2_check(d_x, d_y, n, stream) == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}
+
 int bsattn_debug_trace(int n, int32_t** host_view) {
   if (n < 0 || (n > 0 && !host_view)) return BSATTN_ERR_INVALID_ARG;
 #ifndef BSATTN_TRACE

@@ -71,6 +71,8 @@ struct CombineParams {
 };
 
 cudaError_t launch_build_index(const IndexArgs& a, cudaStream_t stream);
+// y[i] = 2^x[i] through the prefill kernels' FMA-pipe exponential (test hook)
+cudaError_t launch_exp2_check(const float* x, float* y, int64_t n, cudaStream_t stream);
 
 template <int D, int BLK>
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

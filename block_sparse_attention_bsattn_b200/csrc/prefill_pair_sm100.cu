@@ -54,6 +54,14 @@ namespace bsattn {
 // streams at once measured equal or slower.
 constexpr int KVG = 1;
 
+// Exponentials of a kept tile in the variant with the skip vote: of every 8
+// column pairs, the last one goes to the FMA and integer pipes (exp2_fma2)
+// instead of the special-function unit, which the two slots' softmax warps
+// share (1/8 and 2/8 measured best for the BLASST prefill, about 1.6 %
+// faster; 3/8 and 4/8 slower; dense causal attention gained nothing at any
+// share, so the variant without the vote keeps the unit for all of them).
+constexpr int kEmuPairs = 1;
+
 template <int D>
 struct PairCfg {
   static constexpr int BLK = 128;
@@ -517,7 +525,9 @@ __global__ void __launch_bounds__(384, 1)
             for (int c = 0; c < 32; c += 2) {
               const float2 x = ffma2(make_float2(__uint_as_float(r[c0 + c]),
                                                  __uint_as_float(r[c0 + c + 1])), sc2, sh2);
-              const float2 pv = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+              const float2 pv = (VOTE && (c / 2) % 8 >= 8 - kEmuPairs)
+                                    ? exp2_fma2(x)
+                                    : make_float2(fast_exp2(x.x), fast_exp2(x.y));
               rs4[(c / 2) & 3] = fadd2(rs4[(c / 2) & 3], pv);
               pk[c / 2] = pack_bf16x2(pv.x, pv.y);
             }

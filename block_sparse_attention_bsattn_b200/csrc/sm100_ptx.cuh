@@ -319,6 +319,33 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
+// 2^x for two lanes without the special-function unit: x = j + f with
+// j = floor(x) and f in [0, 1) (Cody-Waite style range reduction; adding
+// 1.5 * 2^23 with rounding toward -inf leaves j in the low mantissa bits),
+// 2^f by a cubic fitted on [0, 1) for least maximum relative error (below
+// 9e-5), and j added to the exponent field.  x is clamped below at -127
+// (masked scores of -inf give at most 2^-127, below any bf16 normal).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
+  x.x = fmaxf(x.x, -127.0f);
+  x.y = fmaxf(x.y, -127.0f);
+  float2 t;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
+      "add.rm.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(t.x), "=f"(t.y)
+      : "f"(x.x), "f"(x.y), "f"(kShift));
+  const float2 j = fadd2(t, make_float2(-kShift, -kShift));       // floor(x), exact
+  const float2 f = ffma2(j, make_float2(-1.f, -1.f), x);          // x - j, exact
+  float2 q = ffma2(make_float2(0.07707296f, 0.07707296f), f, make_float2(0.22764768f, 0.22764768f));
+  q = ffma2(q, f, make_float2(0.69511169f, 0.69511169f));
+  q = ffma2(q, f, make_float2(1.f, 1.f));
+  // the low 9 bits of t's pattern hold j (mod 512); shifted by 23 they add j
+  // to q's exponent field
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

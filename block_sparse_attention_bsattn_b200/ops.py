@@ -35,6 +35,8 @@ _lib.bsattn_status_string.restype = ctypes.c_char_p
 _lib.bsattn_version.restype = _I
 _lib.bsattn_debug_set.argtypes = [ctypes.c_longlong, _I]
 _lib.bsattn_debug_set.restype = _I
+_lib.bsattn_debug_exp2.argtypes = [_P, _P, _I64, _P]
+_lib.bsattn_debug_exp2.restype = _I
 _lib.bsattn_debug_trace.argtypes = [_I, ctypes.POINTER(ctypes.POINTER(ctypes.c_int32))]
 _lib.bsattn_debug_trace.restype = _I
 _lib.bsattn_build_index.argtypes = [_P, _I, _I, _I, _I, _I, _I, _P, _P, _I64, _P, _P, _P, _P]
@@ -70,7 +72,8 @@ PREFILL_REVERSE = 0x1
 PREFILL_SKIP_V = 0x2
 DECODE_SINK_SEED = 0x1
 
-EXPORTED = ("bsattn_status_string", "bsattn_version", "bsattn_debug_set", "bsattn_debug_trace",
+EXPORTED = ("bsattn_status_string", "bsattn_version", "bsattn_debug_set", "bsattn_debug_exp2",
+            "bsattn_debug_trace",
             "bsattn_build_index",
             "bsattn_fwd_prefill", "bsattn_fwd_prefill_ex", "bsattn_fwd_prefill_host",
             "bsattn_decode_workspace_size",
@@ -99,6 +102,18 @@ def bsattn_debug_set(wait_limit_ns: int = 2_000_000_000, inject_stall: bool = Fa
     rc = _lib.bsattn_debug_set(int(wait_limit_ns), int(bool(inject_stall)))
     if rc:
         raise BsattnError(rc, "bsattn_debug_set")
+
+
+def bsattn_debug_exp2(x: torch.Tensor) -> torch.Tensor:
+    """Test hook: 2^x through the prefill kernels' FMA-pipe exponential, for
+    a contiguous float32 CUDA tensor."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    rc = _lib.bsattn_debug_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream(None))
+    if rc:
+        raise BsattnError(rc, "bsattn_debug_exp2")
+    return y
 
 
 def bsattn_debug_trace(n: int):

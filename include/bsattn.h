@@ -75,6 +75,18 @@ int bsattn_version(void);
 int bsattn_debug_set(long long wait_limit_ns, int inject_stall);
 
 /*
+ * bsattn_debug_exp2 -- test hook: d_y[i] = 2^d_x[i] for i < n through the
+ * exponential that the prefill kernels run on the FMA and integer pipes for
+ * part of a kept tile's columns (range reduction to floor(x) and a fraction,
+ * a cubic for 2^fraction, the integer part added to the exponent field).
+ * d_x and d_y are device buffers of n floats owned by the caller; the call is
+ * asynchronous on `stream`.  Relative error below 1e-4 for x in [-126, 64);
+ * exactly 0 for x <= -127 and x = -inf.  n < 0, n > 2^32 or a NULL buffer
+ * with n > 0 give BSATTN_ERR_INVALID_ARG.
+ */
+int bsattn_debug_exp2(const float *d_x, float *d_y, int64_t n, cudaStream_t stream);
+
+/*
  * bsattn_debug_trace -- debugging aid, process-wide, present only in a
  * library built with -DBSATTN_TRACE.  The shipped library has no trace
  * markers compiled into its kernels: there n = 0 returns BSATTN_OK (and sets

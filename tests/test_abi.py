@@ -187,3 +187,12 @@ def test_backward_host_validation(lib):
     assert call(q=0x1008) == -3
     assert call(dq=0xb004) == -3
     assert call(wsb=100) == -4          # workspace too small
+
+
+def test_exp2_hook_validation(lib):
+    f = lib.bsattn_debug_exp2
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
+    assert f(None, None, -1, None) == -1
+    assert f(None, 0x1000, 4, None) == -1
+    assert f(0x1000, None, 4, None) == -1
+    assert f(0x1000, 0x2000, (1 << 32) + 1, None) == -1
