@@ -771,7 +771,12 @@ def main():
                     "flops_per_launch": p_flops,
                     "strict_flops_per_launch": strict_flops,
                     "strict_tflops": strict_flops / (p_ms * 1e-3) / 1e12,
-                    "launch_ms": p_ms}
+                    "launch_ms": p_ms,
+                    # context only: the step runs long enough for the board's
+                    # power cap to lower the SM clock, which the burst peak
+                    # does not see; cuBLAS under the same cap sustains this
+                    "frac_of_sustained_peak": tf_rank / peaks["bf16_tflops_sustained"],
+                    "sustained_peak": peaks["bf16_tflops_sustained"]}
     decode_roof = {"kernel": "decode_tc_kernel<128, 4> + decode_combine_kernel",
                    "bound": "hbm", "achieved": gb_rank, "peak": hbm_peak,
                    "unit": "GB/s", "frac": gb_rank / hbm_peak,

@@ -6,6 +6,15 @@
     python -m block_sparse_attention_bsattn_b200.microbench table4
     python -m block_sparse_attention_bsattn_b200.microbench backward --heads 32 --a 10
 
+    python -m block_sparse_attention_bsattn_b200.microbench sustained
+
+`sustained` runs the benchmark's two workloads (the 32-head BLASST prefill
+through a CSR index with its row order, and the 64-sequence decode) back to
+back for about a second per phase -- prefill alone, the index + prefill +
+decode step, the step with an idle gap, decode alone -- with nvidia-smi
+sampling the SM clock and board power, to show what the 1 kW power cap does to
+launches that run longer than a burst.
+
 `table4` sweeps lambda = a / L on the B200 shapes of the BLASST page's Table 4
 (prefill: batch 148, 1 query / 1 KV head, 32K tokens, d 128, causal; decode:
 batch 148, 32 query / 4 KV heads, 32K tokens, d 128) and reports, per a, the
@@ -139,10 +148,89 @@ def backward(args):
             "tflops": 5 * TILE * exe / ms / 1e9, "tflops_issued": 7 * TILE * exe / ms / 1e9}
 
 
+def sustained(args):
+    """Per-phase CUDA-event times with the SM clock and power sampled by
+    nvidia-smi (every 50 ms) over each phase."""
+    import datetime
+    import subprocess
+    import time
+    pw = inputs.workload("blasst_prefill", device="cuda")
+    dw = inputs.workload("blasst_decode", device="cuda")
+    p_lam, d_lam = inputs.lambda_for(args.a, pw.N), inputs.lambda_for(args.a, dw.N)
+    mask = torch.ones(1, pw.nq, pw.nk, dtype=torch.uint8, device="cuda")
+    rp, ci, _, order = ops.bsattn_build_index(mask, 128, 128, True, with_order=True)
+    o, lse = torch.empty_like(pw.q), torch.empty(pw.B, pw.Hq, pw.N, device="cuda")
+    dout, dlse = torch.empty_like(dw.q), torch.empty(dw.B, dw.Hq, device="cuda")
+    ws = torch.empty(ops.bsattn_decode_workspace_size(dw.B, dw.Hq, dw.d, dw.num_splits),
+                     dtype=torch.uint8, device="cuda")
+
+    def index():
+        ops.bsattn_build_index(mask, 128, 128, True, with_order=True)
+
+    def prefill():
+        ops.bsattn_fwd_prefill(pw.q, pw.k, pw.v, 128, pw.scale, True, p_lam, rp, ci, 1, o=o,
+                               lse=lse, row_order=order)
+
+    def decode():
+        ops.bsattn_fwd_decode(dw.q, dw.k, dw.v, 128, dw.num_splits, dw.scale, d_lam, o=dout,
+                              lse=dlse, workspace=ws)
+
+    def idle():
+        torch.cuda._sleep(20_000_000)   # about 10 ms
+
+    prefill(), decode()
+    torch.cuda.synchronize()
+    smi = subprocess.Popen(["nvidia-smi", "--query-gpu=timestamp,clocks.sm,power.draw,"
+                            "clocks_event_reasons.sw_power_cap", "--format=csv,noheader",
+                            "-lms", "50"], stdout=subprocess.PIPE, text=True)
+    phases = [("prefill alone", [prefill], 200), ("step", [index, prefill, decode], 100),
+              ("step + 10 ms idle", [index, prefill, decode, idle], 40),
+              ("decode alone", [decode], 200)]
+    res = []
+    stream = torch.cuda.current_stream()
+    for name, fns, n in phases:
+        idle()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+              for _ in range(n)]
+        t0 = time.time()
+        for i in range(n):
+            ev[i][0].record(stream)
+            for j, f in enumerate(fns):
+                f()
+                ev[i][j + 1].record(stream)
+        torch.cuda.synchronize()
+        t1 = time.time()
+        ms = [[ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(n)] for j in range(len(fns))]
+        res.append({"phase": name, "t": (t0, t1),
+                    "first5_ms": [round(sum(m[:5]) / 5, 3) for m in ms],
+                    "rest_ms": [round(sum(m[n // 4:]) / (n - n // 4), 3) for m in ms]})
+    time.sleep(0.2)
+    smi.terminate()
+    txt, _ = smi.communicate()
+    samples = []
+    for line in txt.strip().splitlines():
+        f = [x.strip() for x in line.split(",")]
+        try:
+            ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            samples.append((ts, float(f[1].split()[0]), float(f[2].split()[0]),
+                            f[3].lower().startswith("active")))
+        except (ValueError, IndexError):
+            continue
+    for r in res:
+        t0, t1 = r.pop("t")
+        sel = [x for x in samples if t0 <= x[0] <= t1]
+        if sel:
+            mhz, watts = sorted(x[1] for x in sel), sorted(x[2] for x in sel)
+            r.update(sm_mhz_median=mhz[len(mhz) // 2], power_w_median=watts[len(watts) // 2],
+                     capped_samples=sum(x[3] for x in sel), samples=len(sel))
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("what", choices=("prefill", "decode", "videodit", "mmdit", "table4",
-                                     "varlen", "backward"))
+                                     "varlen", "backward", "sustained"))
     ap.add_argument("--heads", type=int, default=8, help="query heads (prefill/videodit/mmdit)")
     ap.add_argument("--n", type=int, default=32768, help="sequence length (prefill)")
     ap.add_argument("--batch", type=int, default=64, help="batch (decode)")
@@ -212,6 +300,8 @@ def main():
         out["rows"] = varlen(args)
     elif args.what == "backward":
         out.update(backward(args))
+    elif args.what == "sustained":
+        out["phases"] = sustained(args)
     else:
         B, Hq, Hkv, L, d = args.batch, 32, args.hkv, args.l, 128
         ns = args.splits
