@@ -21,6 +21,10 @@ struct BackwardParams {
   __nv_bfloat16* dv;
   int32_t* status;
   int B, Hq, Hkv, N, nq, nk, d, causal;
+  // causal work order: the lead_k lowest key tiles of every KV head (dK/dV)
+  // and the lead_q last query tiles of every head (dQ) -- the longest work
+  // items, about one wave of them -- go first, all heads at once
+  int lead_k, lead_q;
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
 };

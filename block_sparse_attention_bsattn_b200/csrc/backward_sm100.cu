@@ -25,9 +25,15 @@
 // No atomics: each output tile has one writer.  Warps: 0 TMA producer (it also
 // finds the executed tiles, 32 status bytes per ballot, and passes each one to
 // the other roles through its stage), 1 MMA issuer, 4..11 the element-wise
-// work: two warps per TMEM lane quarter, each owning half of the tile's
+// work: two warps per TMEM lane quarter, each owning half of a half-tile's
 // columns and writing its bf16 results inside them.  Every wait is bounded
 // in time.
+//
+// Each pair (dK/dV) or key tile (dQ) is taken as two halves of 64 columns
+// (queries, resp. keys) with their S and dP in one of two TMEM buffers, so
+// the element-wise work on one half runs while the tensor core computes the
+// other half's products: the first products of half h + 1 are issued before
+// the second products of half h, which wait for its bf16 operands.
 #include <cmath>
 #include <cstdint>
 #include <cuda.h>
@@ -101,16 +107,19 @@ struct BwdCfg {
   // TMEM columns
   static constexpr uint32_t ACC0 = 0;               // dK (dK/dV kernel) or dQ
   static constexpr uint32_t ACC1 = D;               // dV (dK/dV kernel)
-  static constexpr uint32_t S_COL = 256;            // S or S^T, then P^T / dS in bf16
-  static constexpr uint32_t DP_COL = 384;           // dP or dP^T, then dS^T in bf16
+  // half-tile buffer b at BUF + 128 b: S (or S^T) of 64 columns, then its
+  // bf16 P^T / dS at the same place; dP (or dP^T) 64 columns further on, then
+  // dS^T in bf16
+  static constexpr uint32_t BUF = 256;
+  static constexpr uint32_t DPOFF = 64;
   static constexpr int THREADS = 384;              // 4 role warps + 8 element-wise warps
 };
 
 struct BwdBarriers {
   uint64_t res_full;           // resident tiles landed
   uint64_t st_full[2], st_empty[2];
-  uint64_t s_full;             // S and dP of the current pair are in TMEM
-  uint64_t p_ready;            // bf16 operands written back (4 warps)
+  uint64_t s_full[2];          // per half-tile buffer: S and dP are in TMEM
+  uint64_t p_ready[2];         // per buffer: bf16 operands written back (8 warps)
   uint64_t acc_done;           // every MMA finished
   uint64_t drain;
   uint32_t tmem_base;
@@ -118,12 +127,12 @@ struct BwdBarriers {
   int meta[2][2];              // per stage: (head, query tile) / (key tile, -) or -1 = end
 };
 
-// TMEM column (relative to S or dP) of the bf16 pairs of K-step kk (16 of
-// the 128 inner indices) of the element-wise results: the warps that own
-// inner indices [64 h, 64 h + 64) write their 32 columns of pairs at 64 h,
-// inside the 64 fp32 columns they alone read.
+// TMEM column (relative to S or dP of a half-tile buffer) of the bf16 pairs
+// of K-step kk (16 of the half's 64 inner indices) of the element-wise
+// results: the warps that own inner indices [32 h, 32 h + 32) write their 16
+// columns of pairs at 32 h, inside the 32 fp32 columns they alone read.
 __device__ __forceinline__ uint32_t bf16_col(int kk) {
-  return (uint32_t)((kk / 4) * 64 + (kk % 4) * 8);
+  return (uint32_t)((kk / 2) * 32 + (kk % 2) * 8);
 }
 
 // Producer's end-of-stream marker in stage t % 2 (no bytes: a plain arrive).
@@ -151,9 +160,26 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // work item: key tile j of (b, kvh); ascending j first (the longest causal columns)
-  const int bkv = (int)(blockIdx.x / (unsigned)p.nk);
-  const int j = (int)(blockIdx.x - (unsigned)bkv * p.nk);
+  // work item: key tile j of (b, kvh).  Causal: the lead_k lowest key tiles
+  // (the longest columns) of every KV head first, all KV heads at once, so
+  // that no KV head's longest columns start late and run on alone; then each
+  // KV head's remaining tiles in ascending order, KV head by KV head (its
+  // query-side tiles stay in L2 while its CTAs run)
+  int bkv, j;
+  {
+    const int BK = p.B * p.Hkv;
+    const int lead = p.lead_k;
+    const unsigned x = blockIdx.x;
+    if (x < (unsigned)(lead * BK)) {
+      j = (int)(x / (unsigned)BK);
+      bkv = (int)(x - (unsigned)j * BK);
+    } else {
+      const unsigned y = x - (unsigned)(lead * BK);
+      const int rest = p.nk - lead;
+      bkv = (int)(y / (unsigned)rest);
+      j = lead + (int)(y - (unsigned)bkv * rest);
+    }
+  }
   const int b = bkv / p.Hkv, kvh = bkv % p.Hkv;
   const int g = p.Hq / p.Hkv;
   const int len = p.seq_lens ? min(max(p.seq_lens[b], 0), p.N) : p.N;
@@ -164,8 +190,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->st_full[s], 1);
       mbar_init(&bars->st_empty[s], 1);
     }
-    mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->p_ready, 8);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->p_ready[x], 8);
+    }
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -246,49 +274,69 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 1) {
     // ======================================================== MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t k_addr = smem_u32(smem + C::KV_K);
       const uint32_t v_addr = smem_u32(smem + C::KV_V);
-      bool ok = mbar_wait(&bars->res_full, 0, abort, lim);
-      tc_fence_after();
-      for (int t = 0; ok; ++t) {
-        const int st = t & 1;
-        if (!mbar_wait(&bars->st_full[st], (t >> 1) & 1, abort, lim)) break;
-        tc_fence_after();
-        if (*reinterpret_cast<volatile int*>(&bars->meta[st][0]) < 0) break;
-        const uint32_t qa = smem_u32(smem + C::KV_STG + st * C::KV_STG_BYTES);
+      // S^T and dP^T of half x (queries 64 (x & 1) .. + 64 of the pair in
+      // stage st): keys on the rows, the half's queries on the columns
+      auto first = [&](int x, int st) {
+        const uint32_t buf = tmem + C::BUF + 128u * (uint32_t)(x & 1);
+        const uint32_t qa = smem_u32(smem + C::KV_STG + st * C::KV_STG_BYTES) + (x & 1) * 8192;
         const uint32_t da = qa + C::T_BYTES;
-        // S^T = K Q^T and dP^T = V dO^T: keys on the rows, queries on the columns
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(tmem + C::S_COL, smem_desc(k_addr + off, 16, 1024, 2),
-                 smem_desc(qa + off, 16, 1024, 2), IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(buf, smem_desc(k_addr + off, 16, 1024, 2), smem_desc(qa + off, 16, 1024, 2),
+                 IDESC_S, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(tmem + C::DP_COL, smem_desc(v_addr + off, 16, 1024, 2),
+          mma_ss(buf + C::DPOFF, smem_desc(v_addr + off, 16, 1024, 2),
                  smem_desc(da + off, 16, 1024, 2), IDESC_S, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars->s_full);
-        if (!mbar_wait(&bars->p_ready, t & 1, abort, lim)) break;
+        mma_commit(&bars->s_full[x & 1]);
+      };
+      // dV += P^T dO and dK += dS^T Q over half x (scale folded into dS): A
+      // from TMEM, B = the half's rows of the query-side tiles read MN-major;
+      // the stage is released after its second half
+      auto second = [&](int x, int st) -> bool {
+        if (!mbar_wait(&bars->p_ready[x & 1], (x >> 1) & 1, abort, lim)) return false;
         tc_fence_after();
-        // dV += P^T dO and dK += dS^T Q (scale folded into dS): A from TMEM,
-        // B = the query-side tile read MN-major
+        const uint32_t buf = tmem + C::BUF + 128u * (uint32_t)(x & 1);
+        const uint32_t qa = smem_u32(smem + C::KV_STG + st * C::KV_STG_BYTES) + (x & 1) * 8192;
+        const uint32_t da = qa + C::T_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tmem + C::ACC1, tmem + C::S_COL + bf16_col(kk),
+        for (int kk = 0; kk < 64 / 16; ++kk)
+          mma_ts(tmem + C::ACC1, buf + bf16_col(kk),
                  smem_desc(da + kk * (16 * 128), C::T_HALF, 1024, 2), IDESC_O,
-                 (t > 0 || kk > 0) ? 1u : 0u);
+                 (x > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tmem + C::ACC0, tmem + C::DP_COL + bf16_col(kk),
+        for (int kk = 0; kk < 64 / 16; ++kk)
+          mma_ts(tmem + C::ACC0, buf + C::DPOFF + bf16_col(kk),
                  smem_desc(qa + kk * (16 * 128), C::T_HALF, 1024, 2), IDESC_O,
-                 (t > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars->st_empty[st]);
+                 (x > 0 || kk > 0) ? 1u : 0u);
+        if (x & 1) mma_commit(&bars->st_empty[st]);
+        return true;
+      };
+      bool ok = mbar_wait(&bars->res_full, 0, abort, lim);
+      tc_fence_after();
+      int x = 0;   // halves whose first products are issued
+      for (int t = 0; ok; ++t) {
+        const int st = t & 1;
+        if (!mbar_wait(&bars->st_full[st], (t >> 1) & 1, abort, lim)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (*reinterpret_cast<volatile int*>(&bars->meta[st][0]) < 0) break;
+        for (int hh = 0; hh < 2 && ok; ++hh, ++x) {
+          first(x, st);
+          if (x > 0) ok = second(x - 1, hh ? st : st ^ 1);
+        }
       }
+      if (ok && x > 0) second(x - 1, ((x - 1) >> 1) & 1);
       mma_commit(&bars->acc_done);
       mma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0, lim);
@@ -296,8 +344,8 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp >= 4) {
     // ======================================================== element-wise warps
     // Two warps per TMEM lane quarter: warp half hc owns the query columns
-    // [64 hc, 64 hc + 64) of its 32 key rows and writes their bf16 pairs at
-    // column 64 hc, inside the columns only it reads.
+    // [32 hc, 32 hc + 32) of each half-tile for its 32 key rows and writes
+    // their bf16 pairs at column 32 hc, inside the columns only it reads.
     const int quarter = warp % 4;
     const int hc = (warp - 4) / 4;
     const int c = quarter * 32 + lane;           // key row of the tile
@@ -315,24 +363,25 @@ __global__ void __launch_bounds__(384, 1)
       }
       const int ii = *reinterpret_cast<volatile int*>(&bars->meta[st][1]);
       if (*reinterpret_cast<volatile int*>(&bars->meta[st][0]) < 0) break;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, t & 1, abort, lim))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
       const float* lse2 =
           reinterpret_cast<const float*>(smem + C::KV_STG + st * C::KV_STG_BYTES + 2 * C::T_BYTES);
       const float* dvec = lse2 + 128;
-      const int q0 = ii * 128;
       // a query tile after the key tile sees every key (causal), so only the
       // diagonal pair needs the per-element mask
       const bool diag = p.causal && ii == j;
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c0 = 64 * hc + 32 * cc;        // 32 query columns
+      for (int hh = 0; hh < 2 && ok; ++hh) {
+        const int x = 2 * t + hh;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[x & 1], (x >> 1) & 1, abort, lim))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t buf = lane_addr + C::BUF + 128u * (uint32_t)(x & 1);
+        const int c0 = 64 * hh + 32 * hc;          // 32 query columns of the tile
+        const int q0 = ii * 128 + c0;
         uint32_t s[32], dp[32];
-        tmem_ld32(lane_addr + C::S_COL + c0, s);
-        tmem_ld32(lane_addr + C::DP_COL + c0, dp);
+        tmem_ld32(buf + 32 * hc, s);
+        tmem_ld32(buf + C::DPOFF + 32 * hc, dp);
         tmem_wait_ld();
         uint32_t pk[16], dk[16];
 #pragma unroll
@@ -343,13 +392,13 @@ __global__ void __launch_bounds__(384, 1)
           for (int u = 0; u < 4; u += 2) {
             const float2 lu = u == 0 ? make_float2(-l4.x, -l4.y) : make_float2(-l4.z, -l4.w);
             const float2 du = u == 0 ? make_float2(-d4.x, -d4.y) : make_float2(-d4.z, -d4.w);
-            const float2 x = ffma2(make_float2(__uint_as_float(s[r + u]),
-                                               __uint_as_float(s[r + u + 1])), sl2, lu);
-            float2 pv = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            const float2 xv = ffma2(make_float2(__uint_as_float(s[r + u]),
+                                                __uint_as_float(s[r + u + 1])), sl2, lu);
+            float2 pv = make_float2(fast_exp2(xv.x), fast_exp2(xv.y));
             if (!key_ok) pv = make_float2(0.f, 0.f);
             if (diag) {
-              if (key > q0 + c0 + r + u) pv.x = 0.f;
-              if (key > q0 + c0 + r + u + 1) pv.y = 0.f;
+              if (key > q0 + r + u) pv.x = 0.f;
+              if (key > q0 + r + u + 1) pv.y = 0.f;
             }
             const float2 g = fadd2(make_float2(__uint_as_float(dp[r + u]),
                                                __uint_as_float(dp[r + u + 1])), du);
@@ -359,13 +408,14 @@ __global__ void __launch_bounds__(384, 1)
             dk[(r + u) / 2] = pack_bf16x2(ds.x, ds.y);
           }
         }
-        tmem_st16(lane_addr + C::S_COL + 64 * hc + 16 * cc, pk);
-        tmem_st16(lane_addr + C::DP_COL + 64 * hc + 16 * cc, dk);
+        tmem_st16(buf + 32 * hc, pk);
+        tmem_st16(buf + C::DPOFF + 32 * hc, dk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_ready[x & 1]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_ready);
+      if (!ok) break;
     }
     // ---- epilogue: the key tile's dK rows (warp half 0) and dV rows (half 1),
     // zero when no pair took part
@@ -423,9 +473,25 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // work item: query tile i of (b, h); longest causal rows first
-  const int bh = (int)(blockIdx.x / (unsigned)p.nq);
-  const int r = (int)(blockIdx.x - (unsigned)bh * p.nq);
+  // work item: query tile i of (b, h), ranked r (causal: longest rows, the
+  // last query tiles, first).  The lead_q best-ranked rows of every head go
+  // first, all heads at once; then each head's remaining rows in rank order,
+  // head by head
+  int bh, r;
+  {
+    const int BH = p.B * p.Hq;
+    const int lead = p.lead_q;
+    const unsigned x = blockIdx.x;
+    if (x < (unsigned)(lead * BH)) {
+      r = (int)(x / (unsigned)BH);
+      bh = (int)(x - (unsigned)r * BH);
+    } else {
+      const unsigned y = x - (unsigned)(lead * BH);
+      const int rest = p.nq - lead;
+      bh = (int)(y / (unsigned)rest);
+      r = lead + (int)(y - (unsigned)bh * rest);
+    }
+  }
   const int i = p.causal ? p.nq - 1 - r : r;
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int kvh = h / (p.Hq / p.Hkv);
@@ -437,8 +503,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->st_full[s], 1);
       mbar_init(&bars->st_empty[s], 1);
     }
-    mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->p_ready, 8);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->p_ready[x], 8);
+    }
     mbar_init(&bars->acc_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -512,43 +580,62 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 1) {
     // ======================================================== MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q_addr = smem_u32(smem + C::Q_Q);
       const uint32_t do_addr = smem_u32(smem + C::Q_DO);
-      bool ok = mbar_wait(&bars->res_full, 0, abort, lim);
-      tc_fence_after();
-      for (int t = 0; ok; ++t) {
-        const int st = t & 1;
-        if (!mbar_wait(&bars->st_full[st], (t >> 1) & 1, abort, lim)) break;
-        tc_fence_after();
-        if (*reinterpret_cast<volatile int*>(&bars->meta[st][0]) < 0) break;
-        const uint32_t ka = smem_u32(smem + C::Q_STG + st * C::Q_STG_BYTES);
+      // S and dP of half x (keys 64 (x & 1) .. + 64 of the key tile in stage st)
+      auto first = [&](int x, int st) {
+        const uint32_t buf = tmem + C::BUF + 128u * (uint32_t)(x & 1);
+        const uint32_t ka = smem_u32(smem + C::Q_STG + st * C::Q_STG_BYTES) + (x & 1) * 8192;
         const uint32_t va = ka + C::T_BYTES;
-        // S = Q K^T and dP = dO V^T
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(tmem + C::S_COL, smem_desc(q_addr + off, 16, 1024, 2),
-                 smem_desc(ka + off, 16, 1024, 2), IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(buf, smem_desc(q_addr + off, 16, 1024, 2), smem_desc(ka + off, 16, 1024, 2),
+                 IDESC_S, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(tmem + C::DP_COL, smem_desc(do_addr + off, 16, 1024, 2),
+          mma_ss(buf + C::DPOFF, smem_desc(do_addr + off, 16, 1024, 2),
                  smem_desc(va + off, 16, 1024, 2), IDESC_S, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bars->s_full);
-        if (!mbar_wait(&bars->p_ready, t & 1, abort, lim)) break;
+        mma_commit(&bars->s_full[x & 1]);
+      };
+      // dQ += dS K over half x (scale folded into dS): A from TMEM, B = the
+      // half's rows of the K tile read MN-major; the stage is released after
+      // its second half
+      auto second = [&](int x, int st) -> bool {
+        if (!mbar_wait(&bars->p_ready[x & 1], (x >> 1) & 1, abort, lim)) return false;
         tc_fence_after();
-        // dQ += dS K (scale folded into dS): A from TMEM, B = the K tile read MN-major
+        const uint32_t buf = tmem + C::BUF + 128u * (uint32_t)(x & 1);
+        const uint32_t ka = smem_u32(smem + C::Q_STG + st * C::Q_STG_BYTES) + (x & 1) * 8192;
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tmem + C::ACC0, tmem + C::S_COL + bf16_col(kk),
+        for (int kk = 0; kk < 64 / 16; ++kk)
+          mma_ts(tmem + C::ACC0, buf + bf16_col(kk),
                  smem_desc(ka + kk * (16 * 128), C::T_HALF, 1024, 2), IDESC_O,
-                 (t > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars->st_empty[st]);
+                 (x > 0 || kk > 0) ? 1u : 0u);
+        if (x & 1) mma_commit(&bars->st_empty[st]);
+        return true;
+      };
+      bool ok = mbar_wait(&bars->res_full, 0, abort, lim);
+      tc_fence_after();
+      int x = 0;   // halves whose first products are issued
+      for (int t = 0; ok; ++t) {
+        const int st = t & 1;
+        if (!mbar_wait(&bars->st_full[st], (t >> 1) & 1, abort, lim)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (*reinterpret_cast<volatile int*>(&bars->meta[st][0]) < 0) break;
+        for (int hh = 0; hh < 2 && ok; ++hh, ++x) {
+          first(x, st);
+          if (x > 0) ok = second(x - 1, hh ? st : st ^ 1);
+        }
       }
+      if (ok && x > 0) second(x - 1, ((x - 1) >> 1) & 1);
       mma_commit(&bars->acc_done);
       mma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0, lim);
@@ -556,8 +643,8 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp >= 4) {
     // ======================================================== element-wise warps
     // Two warps per TMEM lane quarter: warp half hc owns the key columns
-    // [64 hc, 64 hc + 64) of its 32 query rows and writes their bf16 pairs at
-    // column 64 hc, inside the columns only it reads.
+    // [32 hc, 32 hc + 32) of each half-tile for its 32 query rows and writes
+    // their bf16 pairs at column 32 hc, inside the columns only it reads.
     const int quarter = warp % 4;
     const int hc = (warp - 4) / 4;
     const int rr = quarter * 32 + lane;          // query row of the tile
@@ -579,45 +666,45 @@ __global__ void __launch_bounds__(384, 1)
       }
       const int j = *reinterpret_cast<volatile int*>(&bars->meta[st][0]);
       if (j < 0) break;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, t & 1, abort, lim))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const int k0 = j * 128;
-      // a key tile before the query tile and inside the sequence needs no
-      // per-element mask
-      const bool masked = (p.causal && j == i) || k0 + 128 > len;
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c0 = 64 * hc + 32 * cc;        // 32 key columns
-        uint32_t s[32], dp[32];
-        tmem_ld32(lane_addr + C::S_COL + c0, s);
-        tmem_ld32(lane_addr + C::DP_COL + c0, dp);
+      for (int hh = 0; hh < 2 && ok; ++hh) {
+        const int x = 2 * t + hh;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[x & 1], (x >> 1) & 1, abort, lim))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t buf = lane_addr + C::BUF + 128u * (uint32_t)(x & 1);
+        const int k0 = j * 128 + 64 * hh + 32 * hc;   // first of this warp's 32 keys
+        // keys up to the query and inside the sequence need no per-element mask
+        const bool masked = (p.causal && k0 + 31 > qpos) || k0 + 32 > len;
+        uint32_t sv[32], dp[32];
+        tmem_ld32(buf + 32 * hc, sv);
+        tmem_ld32(buf + C::DPOFF + 32 * hc, dp);
         tmem_wait_ld();
         uint32_t dk[16];
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          const float2 y = ffma2(make_float2(__uint_as_float(s[x]), __uint_as_float(s[x + 1])),
+        for (int xx = 0; xx < 32; xx += 2) {
+          const float2 y = ffma2(make_float2(__uint_as_float(sv[xx]), __uint_as_float(sv[xx + 1])),
                                  sl2, nl2);
           float2 pv = make_float2(fast_exp2(y.x), fast_exp2(y.y));
           if (masked) {
-            const int key = k0 + c0 + x;
+            const int key = k0 + xx;
             if (key >= len || (p.causal && key > qpos)) pv.x = 0.f;
             if (key + 1 >= len || (p.causal && key + 1 > qpos)) pv.y = 0.f;
           }
-          const float2 g = fadd2(make_float2(__uint_as_float(dp[x]), __uint_as_float(dp[x + 1])),
+          const float2 g = fadd2(make_float2(__uint_as_float(dp[xx]), __uint_as_float(dp[xx + 1])),
                                  nd2);
           const float2 ds = ffma2(make_float2(pv.x * p.scale, pv.y * p.scale), g,
                                   make_float2(0.f, 0.f));
-          dk[x / 2] = pack_bf16x2(ds.x, ds.y);
+          dk[xx / 2] = pack_bf16x2(ds.x, ds.y);
         }
-        tmem_st16(lane_addr + C::S_COL + 64 * hc + 16 * cc, dk);
+        tmem_st16(buf + 32 * hc, dk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_ready[x & 1]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_ready);
+      if (!ok) break;
     }
     // ---- epilogue: this query tile's dQ rows, columns [hc D/2, hc D/2 + D/2)
     // per warp half (zero when no key tile took part)

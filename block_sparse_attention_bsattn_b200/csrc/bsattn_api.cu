@@ -422,6 +422,13 @@ int bsattn_bwd_prefill(const void* q, const void* k, const void* v, const void* 
   p.scale = scale;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
   p.wait_limit_ns = g_wait_limit_ns;
+  {
+    const int sms = sm_count();
+    if (sms <= 0) return BSATTN_ERR_CUDA;
+    const int64_t bk = (int64_t)B * Hkv, bh = (int64_t)B * Hq;
+    p.lead_k = causal ? (int)std::min<int64_t>(nq, (sms + bk - 1) / bk) : 0;
+    p.lead_q = causal ? (int)std::min<int64_t>(nq, (sms + bh - 1) / bh) : 0;
+  }
   const cudaError_t e = d == 128 ? launch_backward<128>(tq, tk, tv, tdo, p, stream)
                                  : launch_backward<64>(tq, tk, tv, tdo, p, stream);
   return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
