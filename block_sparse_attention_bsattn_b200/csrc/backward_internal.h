@@ -25,6 +25,7 @@ struct BackwardParams {
   // and the lead_q last query tiles of every head (dQ) -- the longest work
   // items, about one wave of them -- go first, all heads at once
   int lead_k, lead_q;
+  int debug_stall;   // test hook: the resident tiles are never loaded
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
 };

@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(384, 1)
     // ======================================================== producer
     int t = 0;          // pairs issued
     bool ok = true;
-    if (lane == 0) {
+    if (lane == 0 && !p.debug_stall) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmDO);
       mbar_arrive_expect_tx(&bars->res_full, 2 * C::T_BYTES);
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(384, 1)
       if (ok) ok = bwd_end_marker(bars, t, abort, lim);
       if (*abort) {
         // let every copy this thread started land before the CTA can exit
-        mbar_wait_drain(&bars->res_full, 0, lim);
+        if (!p.debug_stall) mbar_wait_drain(&bars->res_full, 0, lim);
         for (int x = (t > 2 ? t - 2 : 0); x < t; ++x)
           mbar_wait_drain(&bars->st_full[x & 1], (x >> 1) & 1, lim);
       }
@@ -526,7 +526,7 @@ __global__ void __launch_bounds__(384, 1)
     // ======================================================== producer
     int t = 0;
     bool ok = true;
-    if (lane == 0) {
+    if (lane == 0 && !p.debug_stall) {
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
       mbar_arrive_expect_tx(&bars->res_full, 2 * C::T_BYTES);
@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       if (ok) ok = bwd_end_marker(bars, t, abort, lim);
       if (*abort) {
-        mbar_wait_drain(&bars->res_full, 0, lim);
+        if (!p.debug_stall) mbar_wait_drain(&bars->res_full, 0, lim);
         for (int x = (t > 2 ? t - 2 : 0); x < t; ++x)
           mbar_wait_drain(&bars->st_full[x & 1], (x >> 1) & 1, lim);
       }

@@ -429,6 +429,7 @@ int bsattn_bwd_prefill(const void* q, const void* k, const void* v, const void* 
     p.lead_k = causal ? (int)std::min<int64_t>(nq, (sms + bk - 1) / bk) : 0;
     p.lead_q = causal ? (int)std::min<int64_t>(nq, (sms + bh - 1) / bh) : 0;
   }
+  p.debug_stall = g_inject_stall;
   const cudaError_t e = d == 128 ? launch_backward<128>(tq, tk, tv, tdo, p, stream)
                                  : launch_backward<64>(tq, tk, tv, tdo, p, stream);
   return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;

@@ -68,8 +68,9 @@ int bsattn_version(void);
  * pipeline wait inside the kernels (default 2 s); when one runs out the kernel
  * stops, drains its own copies, frees its tensor memory and reports
  * BSATTN_ERR_DEVICE_TIMEOUT through d_status.  inject_stall != 0 makes the
- * prefill kernels withhold their query tile from the tensor core so that the
- * limit is reached on purpose.  Returns BSATTN_ERR_INVALID_ARG for
+ * prefill kernels withhold their query tile from the tensor core, and the
+ * backward kernels their resident tiles, so that the limit is reached on
+ * purpose.  Returns BSATTN_ERR_INVALID_ARG for
  * wait_limit_ns <= 0.
  */
 int bsattn_debug_set(long long wait_limit_ns, int inject_stall);
