@@ -1,7 +1,7 @@
 // Thin inline-PTX wrappers for the sm_100a features the kernels use:
 // mbarriers (with bounded waits), TMA tensor and bulk copies, and the
 // 5th-generation tensor core (tcgen05: TMEM alloc, MMA, commit, ld/st).
-// No cluster multicast form of any copy is used anywhere in this library.
+// Every copy here goes to the issuing CTA's own shared memory only.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
