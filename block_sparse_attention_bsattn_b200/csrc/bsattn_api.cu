@@ -291,10 +291,8 @@ int bsattn_fwd_decode_ex(const void* q, const void* k, const void* v, void* o, f
   if (d != 64 && d != 128) return BSATTN_ERR_UNSUPPORTED;
   if (block != 64 && block != 128) return BSATTN_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
-  // block 128: tensor-core kernel, any group of up to 16 query heads;
-  // block 64: CUDA-core kernel, groups of 1, 2, 4 or 8
-  if (block == 128 ? G > 16 : (G != 1 && G != 2 && G != 4 && G != 8))
-    return BSATTN_ERR_UNSUPPORTED;
+  // the tensor-core kernel takes any group of up to 16 query heads
+  if (G > 16) return BSATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(workspace))
     return BSATTN_ERR_ALIGNMENT;
   if (workspace_bytes < bsattn_decode_workspace_size(B, Hq, d, num_splits))
@@ -336,30 +334,14 @@ int bsattn_fwd_decode_ex(const void* q, const void* k, const void* v, void* o, f
   p.trace = g_trace;
   p.trace_n = g_trace_n;
 
-  cudaError_t e = cudaErrorInvalidValue;
-  if (block == 128) {
-    CUtensorMap tq;
-    if (!encode_bf16_3d(&tq, q, d, Hq, (uint64_t)B, 16)) return BSATTN_ERR_CUDA;
-    const int sms = sm_count();
-    if (sms <= 0) return BSATTN_ERR_CUDA;
-    const int tc_grid = (int)(grid < sms ? grid : sms);
-    e = d == 128 ? launch_decode_tc<128>(tq, tk, tv, p, G, tc_grid, stream)
-                 : launch_decode_tc<64>(tq, tk, tv, p, G, tc_grid, stream);
-    if (e != cudaSuccess) return BSATTN_ERR_CUDA;
-    CombineParams c{p.ws_o, p.ws_m, p.ws_l, static_cast<__nv_bfloat16*>(o), lse, num_splits, d};
-    e = launch_decode_combine(c, B * Hq, d, stream);
-    return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
-  }
-#define BSATTN_DEC(DD, BB, GG)                                               \
-  if (d == DD && block == BB && G == GG)                                     \
-    e = launch_decode_split<DD, BB, GG>(tk, tv, p, (int)grid, stream);
-  BSATTN_DEC(128, 128, 1) BSATTN_DEC(128, 128, 2) BSATTN_DEC(128, 128, 4) BSATTN_DEC(128, 128, 8)
-  BSATTN_DEC(64, 128, 1) BSATTN_DEC(64, 128, 2) BSATTN_DEC(64, 128, 4) BSATTN_DEC(64, 128, 8)
-  BSATTN_DEC(128, 64, 1) BSATTN_DEC(128, 64, 2) BSATTN_DEC(128, 64, 4) BSATTN_DEC(128, 64, 8)
-  BSATTN_DEC(64, 64, 1) BSATTN_DEC(64, 64, 2) BSATTN_DEC(64, 64, 4) BSATTN_DEC(64, 64, 8)
-#undef BSATTN_DEC
+  CUtensorMap tq;
+  if (!encode_bf16_3d(&tq, q, d, Hq, (uint64_t)B, 16)) return BSATTN_ERR_CUDA;
+  const int sms = sm_count();
+  if (sms <= 0) return BSATTN_ERR_CUDA;
+  const int tc_grid = (int)(grid < sms ? grid : sms);
+  cudaError_t e = d == 128 ? launch_decode_tc<128>(tq, tk, tv, p, G, block, tc_grid, stream)
+                           : launch_decode_tc<64>(tq, tk, tv, p, G, block, tc_grid, stream);
   if (e != cudaSuccess) return BSATTN_ERR_CUDA;
-
   CombineParams c{p.ws_o, p.ws_m, p.ws_l, static_cast<__nv_bfloat16*>(o), lse, num_splits, d};
   e = launch_decode_combine(c, B * Hq, d, stream);
   return e == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;

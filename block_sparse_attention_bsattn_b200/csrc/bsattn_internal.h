@@ -83,13 +83,10 @@ cudaError_t launch_prefill_pair(const CUtensorMap& tq, const CUtensorMap& tk,
                                 const CUtensorMap& tv, const PrefillParams& p, int grid,
                                 cudaStream_t stream);
 
-template <int D, int BLK, int G>
-cudaError_t launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv,
-                                const DecodeParams& p, int grid, cudaStream_t stream);
-
 template <int D>
 cudaError_t launch_decode_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const DecodeParams& p, int G, int grid, cudaStream_t stream);
+                             const DecodeParams& p, int G, int block, int grid,
+                             cudaStream_t stream);
 
 cudaError_t launch_decode_combine(const CombineParams& p, int grid, int threads,
                                   cudaStream_t stream);

@@ -30,6 +30,10 @@
 // The exponent shift is lazy: it moves only when the running max exceeds it by
 // more than TAU (base 2); O^T and the row sums are then rescaled after every
 // earlier P.V has completed.  Every wait is bounded in time.
+// Key tiles of 64 tokens (KT = 64) use the same 128-row products: the tile
+// fills rows 0..63 of its K buffer, the scores of rows 64..127 are ignored,
+// and BMM2 runs over the tile's 64 keys only (4 K-steps), so no stale row
+// of a V buffer is ever read.
 // The softmax warps' per-column loops run over NC columns, g rounded up to a
 // power of two and fixed at compile time (one instance per NC), and the
 // per-warp tile max is a butterfly reduce-scatter.  Options: sink-seeded
@@ -46,24 +50,25 @@
 
 namespace bsattn {
 
-template <int D>
+template <int D, int KT>
 struct DecTcCfg {
-  static constexpr int BLK = 128;                 // keys per tile = MMA rows
+  static constexpr int BLK = 128;                 // MMA rows of BMM2 (output dims, padded)
   static constexpr int NQ = 16;                   // MMA N: query columns
   static constexpr int KST = 3;                   // K ring
-  static constexpr int VST = 3;                   // V ring
+  // V ring: with 64-token tiles two stages, so that two CTAs fit on an SM
+  static constexpr int VST = KT == 64 ? 2 : 3;
   static constexpr int LA = 3;                    // BMM1 look-ahead (tiles)
   static constexpr int NS = LA + 1;               // S buffers in TMEM
   static constexpr int PB = 4;                    // P^T slots
   static constexpr int R = 8;                     // BMM2 completion ring (> PB)
   static constexpr int DQ = 8;                    // decision queue to the V producer
   static constexpr int HALVES = D / 64;
-  static constexpr int T_HALF = BLK * 128;        // one 64-column box of a tile
+  static constexpr int T_HALF = KT * 128;         // one 64-column box of a tile
   static constexpr int T_BYTES = HALVES * T_HALF;
   static constexpr int Q_HALF = NQ * 128;         // 16 rows x 128 bytes
   static constexpr int Q_BYTES = HALVES * Q_HALF;
   static constexpr int P_HALF = NQ * 128;         // P^T: 16 rows x 64 keys
-  static constexpr int P_BYTES = 2 * P_HALF;      // 128 keys
+  static constexpr int P_BYTES = (KT / 64) * P_HALF;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + KST * T_BYTES;
   static constexpr int Q_OFF = V_OFF + VST * T_BYTES;
@@ -100,11 +105,15 @@ struct DecTcBarriers {
 // NC: the query columns the softmax warps work on, G rounded up to a power of
 // two, fixed at compile time so that the per-column work of the scores (the
 // reduction, the vote, the exponentials) unrolls and interleaves
-template <int D, int NC>
-__global__ void __launch_bounds__(224, 1)
+// With 64-token tiles and at most 8 query columns two CTAs share an SM
+// (launch bounds cap the registers at 146 per thread).
+template <int D, int NC, int KT>
+__global__ void __launch_bounds__(224, (KT == 64 && NC <= 8) ? 2 : 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const DecodeParams p, int G) {
-  using C = DecTcCfg<D>;
+  using C = DecTcCfg<D, KT>;
+  static_assert(KT == 64 || KT == 128, "key tile");
+  constexpr int KT_BYTES = C::T_BYTES;             // bytes of one K or V tile
   static_assert(NC == 1 || NC == 2 || NC == 4 || NC == 8 || NC == 16, "columns");
   constexpr int LOG_NC = NC >= 16 ? 4 : NC >= 8 ? 3 : NC >= 4 ? 2 : NC >= 2 ? 1 : 0;
   static_assert(sizeof(DecTcBarriers) <= C::BAR_BYTES, "barrier block");
@@ -167,7 +176,7 @@ __global__ void __launch_bounds__(224, 1)
     kvh = bk % p.Hkv;
     int T = p.T, chunk = p.chunk;
     if (p.seq_lens) {
-      T = (len_of(b) + C::BLK - 1) / C::BLK;
+      T = (len_of(b) + KT - 1) / KT;
       chunk = T > 0 ? (T + p.splits - 1) / p.splits : 1;
     }
     t0 = split * chunk;
@@ -197,10 +206,10 @@ __global__ void __launch_bounds__(224, 1)
         for (int t = 0; t < nt; ++t, ++g) {
           const int ks = g % C::KST;
           if (!mbar_wait(&bars->k_empty[ks], ((g / C::KST) & 1) ^ 1, abort, lim)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars->k_full[ks], C::T_BYTES);
+          mbar_arrive_expect_tx(&bars->k_full[ks], KT_BYTES);
           for (int hf = 0; hf < C::HALVES; ++hf)
             tma_load_3d(k_smem + ks * C::T_BYTES + hf * C::T_HALF, &tmK, &bars->k_full[ks],
-                        hf * 64, tile_of(t0, sd, t) * C::BLK, b * p.Hkv + kvh);
+                        hf * 64, tile_of(t0, sd, t) * KT, b * p.Hkv + kvh);
         }
       }
       if (*abort) {
@@ -225,10 +234,10 @@ __global__ void __launch_bounds__(224, 1)
           if (!keep) continue;
           const int vs = kept % C::VST;
           if (!mbar_wait(&bars->v_empty[vs], ((kept / C::VST) & 1) ^ 1, abort, lim)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
+          mbar_arrive_expect_tx(&bars->v_full[vs], KT_BYTES);
           for (int hf = 0; hf < C::HALVES; ++hf)
             tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
-                        hf * 64, tile_of(t0, sd, t) * C::BLK, b * p.Hkv + kvh);
+                        hf * 64, tile_of(t0, sd, t) * KT, b * p.Hkv + kvh);
           ++kept;
         }
       }
@@ -240,7 +249,9 @@ __global__ void __launch_bounds__(224, 1)
   } else if (warp == 1) {
     // ======================================================== MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC1 = idesc_bf16_f32(128, C::NQ, 0, 0);
+      // BMM1 has one MMA row per key: M = 64 for 64-token tiles, whose
+      // accumulator rows 16 q + i (i < 16) sit in TMEM lane 32 q + i
+      constexpr uint32_t IDESC1 = idesc_bf16_f32(KT, C::NQ, 0, 0);
       constexpr uint32_t IDESC2 = idesc_bf16_f32(128, C::NQ, 1, 0);
       const uint32_t k_addr = smem_u32(k_smem), v_addr = smem_u32(v_smem);
       const uint32_t q_addr = smem_u32(q_smem), p_addr = smem_u32(p_smem);
@@ -300,7 +311,7 @@ __global__ void __launch_bounds__(224, 1)
           tc_fence_after();
           const uint32_t o_tmem = tmem + C::O_COL + (n & 1) * 16;
 #pragma unroll
-          for (int kk = 0; kk < C::BLK / 16; ++kk) {
+          for (int kk = 0; kk < KT / 16; ++kk) {
             const uint32_t a = v_addr + vs * C::T_BYTES + kk * (16 * 128);
             const uint32_t bp = p_addr + ps * C::P_BYTES + (kk / 4) * C::P_HALF + (kk % 4) * 32;
             mma_ss(o_tmem, smem_desc(a, D == 128 ? C::T_HALF : 0, 1024, 2),
@@ -320,7 +331,10 @@ __global__ void __launch_bounds__(224, 1)
     // ======================================================== score / softmax warps
     const int sw = warp - 2;                      // 0..3 -> TMEM lane quarter (warp % 4)
     const int quarter = warp % 4;
-    const int key = quarter * 32 + lane;          // key row inside the tile
+    const int row = quarter * 32 + lane;          // TMEM lane
+    // key of the tile in this lane (BMM1 row): with 64-token tiles lanes
+    // 16..31 of each quarter hold no key (KT marks them)
+    const int key = KT == 128 ? row : (lane < 16 ? quarter * 16 + lane : KT);
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const float thr = p.thr_log2;
     int g = 0, kept = 0;
@@ -354,7 +368,7 @@ __global__ void __launch_bounds__(224, 1)
         if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
         const int jt = tile_of(t0, sd, t);
         const bool seed = sd && t == 0;
-        const bool key_ok = jt * C::BLK + key < lenb;
+        const bool key_ok = key < KT && jt * KT + key < lenb;
         float s[NC];
 #pragma unroll
         for (int c = 0; c < NC; ++c) s[c] = (key_ok && c < G) ? __uint_as_float(r[c]) : -INFINITY;
@@ -456,14 +470,16 @@ __global__ void __launch_bounds__(224, 1)
           }
           // P^T[c][key] = exp2(S * scale_log2 - shift) as bf16, 128-byte swizzle
           uint8_t* ps = p_smem + (kept % C::PB) * C::P_BYTES + (key / 64) * C::P_HALF;
+          if (key < KT) {   // a lane without a key writes nothing
 #pragma unroll
-          for (int c = 0; c < NC; ++c) {
-            const float sh = m_ref[c] == -INFINITY ? 0.f : m_ref[c];
-            const float pv = fast_exp2(fmaf(s[c], p.scale_log2, -sh));
-            lp[c] += pv;
-            const int kk = key % 64;
-            *reinterpret_cast<__nv_bfloat16*>(ps + c * 128 + ((((kk >> 3) ^ (c & 7))) << 4) +
-                                              (kk & 7) * 2) = __float2bfloat16_rn(pv);
+            for (int c = 0; c < NC; ++c) {
+              const float sh = m_ref[c] == -INFINITY ? 0.f : m_ref[c];
+              const float pv = fast_exp2(fmaf(s[c], p.scale_log2, -sh));
+              lp[c] += pv;
+              const int kk = key % 64;
+              *reinterpret_cast<__nv_bfloat16*>(ps + c * 128 + ((((kk >> 3) ^ (c & 7))) << 4) +
+                                                (kk & 7) * 2) = __float2bfloat16_rn(pv);
+            }
           }
           fence_proxy_async_smem();
           ++kept;
@@ -512,7 +528,7 @@ __global__ void __launch_bounds__(224, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->epi_full[n & 1]);
       const int64_t base = ((int64_t)b * p.Hq + (int64_t)kvh * G) * p.splits + split;
-      const int dim = key;                         // O^T lane = output dimension
+      const int dim = row;                         // O^T lane = output dimension
       if (dim < D) {
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
@@ -549,32 +565,50 @@ __global__ void __launch_bounds__(224, 1)
   }
 }
 
-template <int D, int NC>
+template <int D, int NC, int KT>
 static cudaError_t launch_decode_tc_nc(const CUtensorMap& tq, const CUtensorMap& tk,
                                        const CUtensorMap& tv, const DecodeParams& p, int G, int grid,
                                        cudaStream_t stream) {
-  using C = DecTcCfg<D>;
+  using C = DecTcCfg<D, KT>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, NC>,
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, NC, KT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  decode_tc_kernel<D, NC><<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p, G);
+  e = cudaFuncSetAttribute(decode_tc_kernel<D, NC, KT>,
+                           cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return e;
+  // `grid` is one CTA per SM (or fewer items); with 64-token tiles and at
+  // most 8 query columns two CTAs per SM (their shared memory, registers
+  // under the launch bounds and 2 x 128 TMEM columns fit).  CTAs never wait
+  // for one another, so a CTA that found no room would simply start later.
+  const int n_items = p.B * p.Hkv * p.splits;
+  if (KT == 64 && NC <= 8) grid = grid * 2 < n_items ? grid * 2 : n_items;
+  decode_tc_kernel<D, NC, KT><<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p, G);
   return cudaGetLastError();
+}
+
+template <int D, int KT>
+static cudaError_t launch_decode_tc_kt(const CUtensorMap& tq, const CUtensorMap& tk,
+                                       const CUtensorMap& tv, const DecodeParams& p, int G, int grid,
+                                       cudaStream_t stream) {
+  if (G <= 1) return launch_decode_tc_nc<D, 1, KT>(tq, tk, tv, p, G, grid, stream);
+  if (G <= 2) return launch_decode_tc_nc<D, 2, KT>(tq, tk, tv, p, G, grid, stream);
+  if (G <= 4) return launch_decode_tc_nc<D, 4, KT>(tq, tk, tv, p, G, grid, stream);
+  if (G <= 8) return launch_decode_tc_nc<D, 8, KT>(tq, tk, tv, p, G, grid, stream);
+  return launch_decode_tc_nc<D, 16, KT>(tq, tk, tv, p, G, grid, stream);
 }
 
 template <int D>
 cudaError_t launch_decode_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const DecodeParams& p, int G, int grid, cudaStream_t stream) {
-  if (G <= 1) return launch_decode_tc_nc<D, 1>(tq, tk, tv, p, G, grid, stream);
-  if (G <= 2) return launch_decode_tc_nc<D, 2>(tq, tk, tv, p, G, grid, stream);
-  if (G <= 4) return launch_decode_tc_nc<D, 4>(tq, tk, tv, p, G, grid, stream);
-  if (G <= 8) return launch_decode_tc_nc<D, 8>(tq, tk, tv, p, G, grid, stream);
-  return launch_decode_tc_nc<D, 16>(tq, tk, tv, p, G, grid, stream);
+                             const DecodeParams& p, int G, int block, int grid,
+                             cudaStream_t stream) {
+  return block == 64 ? launch_decode_tc_kt<D, 64>(tq, tk, tv, p, G, grid, stream)
+                     : launch_decode_tc_kt<D, 128>(tq, tk, tv, p, G, grid, stream);
 }
 
 template cudaError_t launch_decode_tc<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                           const DecodeParams&, int, int, cudaStream_t);
+                                           const DecodeParams&, int, int, int, cudaStream_t);
 template cudaError_t launch_decode_tc<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                          const DecodeParams&, int, int, cudaStream_t);
+                                          const DecodeParams&, int, int, int, cudaStream_t);
 
 }  // namespace bsattn

@@ -237,6 +237,7 @@ def main():
     ap.add_argument("--l", type=int, default=131072, help="KV length (decode)")
     ap.add_argument("--hkv", type=int, default=8, help="KV heads (decode; 32 query heads)")
     ap.add_argument("--splits", type=int, default=16, help="KV splits (decode)")
+    ap.add_argument("--block", type=int, default=128, help="key tile (decode): 64 or 128")
     ap.add_argument("--a", type=float, default=10.0)
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=2)
@@ -307,21 +308,23 @@ def main():
         ns = args.splits
         q, k, v = inputs.blasst_decode_qkv(B, Hq, Hkv, L, d, "cuda", 1238)
         lam = inputs.lambda_for(args.a, L)
-        T = -(-L // 128)
+        blk = args.block
+        T = -(-L // blk)
         st = torch.zeros(B, Hkv, T, dtype=torch.uint8, device="cuda")
         ws = torch.empty(ops.bsattn_decode_workspace_size(B, Hq, d, ns), dtype=torch.uint8,
                          device="cuda")
-        o, _ = ops.bsattn_fwd_decode(q, k, v, 128, ns, None, lam, workspace=ws, tile_status=st,
+        o, _ = ops.bsattn_fwd_decode(q, k, v, blk, ns, None, lam, workspace=ws, tile_status=st,
                                      sink_seed=args.sink_seed)
         torch.cuda.synchronize()
         vis, exe = int((st > 0).sum()), int((st == 2).sum())
-        fn = lambda: ops.bsattn_fwd_decode(q, k, v, 128, ns, None, lam, o=o, want_lse=False,
+        fn = lambda: ops.bsattn_fwd_decode(q, k, v, blk, ns, None, lam, o=o, want_lse=False,
                                            workspace=ws, sink_seed=args.sink_seed)
         for _ in range(args.warmup):
             fn()
         ms = _time(fn, args.iters)
-        byt = 2 * B * Hq * d * 2 + 128 * d * 2 * (vis + exe)
-        out.update(batch=B, l=L, hkv=Hkv, splits=ns, sink_seed=args.sink_seed, a=args.a, visited=vis, executed=exe, ms=ms, gbs=byt / ms / 1e6)
+        byt = 2 * B * Hq * d * 2 + blk * d * 2 * (vis + exe)
+        out.update(batch=B, l=L, hkv=Hkv, splits=ns, block=blk, sink_seed=args.sink_seed, a=args.a,
+                   visited=vis, executed=exe, ms=ms, gbs=byt / ms / 1e6)
     print(json.dumps(out), flush=True)
 
 

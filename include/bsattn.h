@@ -94,7 +94,7 @@ int bsattn_debug_exp2(const float *d_x, float *d_y, int64_t n, cudaStream_t stre
  * *host_view to NULL when given), n > 0 returns BSATTN_ERR_UNSUPPORTED and
  * allocates nothing.  In a trace build, n > 0 allocates n int32 of mapped,
  * pinned host memory (zeroed), returns its host address in *host_view and
- * makes the prefill and decode kernels record progress there, readable while
+ * makes the one-query-tile prefill kernel record progress there, readable while
  * a kernel is still running: slot 16 + CTA index holds the stage a CTA reached
  * (1 entered, 2 set up, 3 finished, 4 tensor memory freed; 13/14 the same
  * after a timed-out wait), slots 8..17 the warps of CTA 0 that have left
@@ -270,8 +270,8 @@ size_t bsattn_decode_workspace_size(int B, int Hq, int d, int num_splits);
  *               bytes, 16-byte aligned, owned by the caller
  *   tile_status uint8 [B][Hkv][T] or NULL (cleared, then 1 skipped / 2 executed)
  *
- * Supported GQA groups Hq/Hkv: 1..16 with block 128 (tensor-core kernel),
- * 1, 2, 4 or 8 with block 64; anything else gives BSATTN_ERR_UNSUPPORTED.
+ * Supported GQA groups Hq/Hkv: 1..16, with key tiles of 64 or 128 tokens
+ * (one tensor-core kernel); anything else gives BSATTN_ERR_UNSUPPORTED.
  */
 int bsattn_fwd_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B,
                       int Hq, int Hkv, int L, int d, int block, float scale, int causal,

@@ -88,7 +88,7 @@ def test_decode_host_validation(lib):
     assert dec(splits=0) == -1
     assert dec(lam=2.0) == -1
     assert dec(Hq=34, Hkv=2) == -2                   # GQA group of 17
-    assert dec(Hq=32, Hkv=2, block=64) == -2         # group of 16 with 64-token tiles
+    assert dec(Hq=34, Hkv=2, block=64) == -2         # group of 17 with 64-token tiles
     assert dec(d=80) == -2
     assert dec(q=0x1004) == -3
     assert dec(wsb=16) == -4                         # workspace too small

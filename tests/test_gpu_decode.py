@@ -67,7 +67,8 @@ def test_decode_operating_point_shrunk():
 @pytest.mark.parametrize("d,block,g", [(64, 64, 1), (64, 128, 2), (128, 64, 8), (128, 128, 4),
                                        (128, 128, 8), (128, 128, 3), (64, 128, 16),
                                        (128, 128, 1), (128, 128, 16), (128, 128, 5),
-                                       (64, 128, 6), (128, 128, 12)])
+                                       (64, 128, 6), (128, 128, 12), (128, 64, 16),
+                                       (64, 64, 3), (128, 64, 5), (64, 64, 12)])
 @pytest.mark.parametrize("splits", [1, 3, 7])
 def test_decode_shapes(d, block, g, splits):
     B, Hkv, L = 2, 2, 5 * block + 19
