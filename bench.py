@@ -777,10 +777,10 @@ def main():
                     # does not see; cuBLAS under the same cap sustains this
                     "frac_of_sustained_peak": tf_rank / peaks["bf16_tflops_sustained"],
                     "sustained_peak": peaks["bf16_tflops_sustained"]}
-    decode_roof = {"kernel": "decode_tc_kernel<128, 4> + decode_combine_kernel",
+    decode_roof = {"kernel": "decode_tc_kernel<128, 4, 128> + decode_combine_kernel",
                    "bound": "hbm", "achieved": gb_rank, "peak": hbm_peak,
                    "unit": "GB/s", "frac": gb_rank / hbm_peak,
-                   "traffic": profiled_traffic("decode_tc_kernel<128, 4>"),
+                   "traffic": profiled_traffic("decode_tc_kernel<128, 4, 128>"),
                    "peak_source": f"{peak_src} copy bandwidth",
                    "bytes_per_launch": d_bytes, "launch_ms": d_ms}
     # the top-level roofline is the one of the kernel that takes the larger
