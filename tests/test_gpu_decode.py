@@ -158,3 +158,15 @@ def test_blasst_decode_full_size_sampled(a):
     pairs = sorted({(int(rng.integers(w.B)), int(rng.integers(w.Hkv))) for _ in range(8)})
     _check(w.q, w.k, w.v, w.block, w.num_splits, w.scale, inputs.lambda_for(a, w.N), pairs,
            what=f"full a={a}")
+
+
+@pytest.mark.parametrize("lam", [1.0, 1e-30])
+@pytest.mark.parametrize("block", [64, 128])
+def test_decode_lambda_at_the_ends_of_its_range(lam, block):
+    """lambda = 1 (a tile is skipped unless some query head reaches the
+    running max) and lambda = 1e-30 (effectively no skipping)."""
+    B, Hkv, g, L = 2, 2, 4, 9 * block + 11
+    q, k, v = inputs.blasst_decode_qkv(B, Hkv * g, Hkv, L, 128, "cpu", 71 + block)
+    ref = _check(q, k, v, block, 3, 1 / math.sqrt(128), lam, what=f"lambda {lam} b{block}")
+    if lam == 1.0:
+        assert (ref["status"] == 1).sum() > 0

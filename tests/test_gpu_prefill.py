@@ -397,3 +397,26 @@ def test_masks_rows_of_their_own(d, causal, lam, per_head):
     rows = slice(3 * 128, 4 * 128)
     assert (o[:, :, rows].float() == 0).all()
     assert torch.isneginf(lse[:, :, rows]).all()
+
+
+@pytest.mark.parametrize("lam", [1.0, 1e-30])
+@pytest.mark.parametrize("hq,hkv,block,masked", [(4, 2, 128, False), (2, 2, 64, False),
+                                                 (3, 3, 128, True)])
+def test_lambda_at_the_ends_of_its_range(lam, hq, hkv, block, masked):
+    """lambda = 1 (the largest allowed: a tile is skipped unless some row
+    reaches the running max) and lambda = 1e-30 (effectively no skipping), on
+    the two-tile kernel, 64-token tiles and a shared mask with one query head
+    per KV head."""
+    N = 5 * block + 23
+    nb = -(-N // block)
+    q, k, v = inputs.blasst_prefill_qkv(1, hq, hkv, N, 128, "cpu", 61 + block)
+    w = inputs.Workload("ends", 1, hq, hkv, N, 128, block, True, "prefill", 1 / math.sqrt(128),
+                        None, q=q, k=k, v=v)
+    mask = None
+    if masked:
+        rng = np.random.default_rng(62)
+        mask = (rng.random((1, nb, nb)) < 0.7).astype(np.uint8)
+        mask[:, np.arange(nb), np.arange(nb)] = 1
+    ref = _check(w, lam, mask, f"lambda {lam} h{hq}/{hkv} b{block}")
+    if lam == 1.0:
+        assert (ref["status"] == 1).sum() > 0
