@@ -123,37 +123,49 @@ int bsattn_fwd_prefill_host(const void* h_q, const void* h_k, const void* h_v, v
       cudaStreamWaitEvent(pipe->out, pipe->start, 0) != cudaSuccess)
     return fail(BSATTN_ERR_CUDA);
 
+  // One KV head per chunk (the finest setting) with an even group of at least
+  // 4 query heads: the first and the last chunk go in pieces of 2 query
+  // heads (the first piece brings the KV head's K and V), so that the first
+  // kernel starts after a smaller copy and the last copy out follows a
+  // smaller kernel -- the copies in set the pace, and these two ends are the
+  // part of the call they cannot hide.
+  const bool split_ends = hkc == 1 && G % 2 == 0 && G >= 4;
   int c = 0;
   for (int b = 0; b < B; ++b) {
-    for (int kv0 = 0; kv0 < Hkv; kv0 += hkc, ++c) {
-      const int hq0 = kv0 * G;
-      const size_t qoff = ((size_t)b * Hq + hq0) * row, qlen = (size_t)hqc * row;
-      const size_t koff = ((size_t)b * Hkv + kv0) * row, klen = (size_t)hkc * row;
-      cudaEvent_t copied = pipe->copied[c % kEvents], computed = pipe->computed[c % kEvents];
-      if (cudaMemcpyAsync(atw(d_q, qoff), at(h_q, qoff), qlen, cudaMemcpyHostToDevice,
-                          pipe->in) != cudaSuccess ||
-          cudaMemcpyAsync(atw(d_k, koff), at(h_k, koff), klen, cudaMemcpyHostToDevice,
-                          pipe->in) != cudaSuccess ||
-          cudaMemcpyAsync(atw(d_v, koff), at(h_v, koff), klen, cudaMemcpyHostToDevice,
-                          pipe->in) != cudaSuccess ||
-          cudaEventRecord(copied, pipe->in) != cudaSuccess ||
-          cudaStreamWaitEvent(stream, copied, 0) != cudaSuccess)
-        return fail(BSATTN_ERR_CUDA);
-      // the chunk as a problem of its own: one sequence, hqc query heads;
-      // per-head CSR rows and orders start at the chunk's first head
-      const bool per_head = row_ptr && mask_heads == Hq;
-      const int rc = bsattn_fwd_prefill(
-          at(d_q, qoff), at(d_k, koff), at(d_v, koff), atw(d_o, qoff), nullptr, 1, hqc, hkc, N, d,
-          block, scale, causal, lambda,
-          row_ptr ? row_ptr + (per_head ? (size_t)hq0 * (nq + 1) : 0) : nullptr, col_idx,
-          row_order ? row_order + (per_head ? (size_t)hq0 * nq : 0) : nullptr,
-          per_head ? hqc : 1, nullptr, d_status, stream);
-      if (rc != BSATTN_OK) return fail(rc);
-      if (cudaEventRecord(computed, stream) != cudaSuccess ||
-          cudaStreamWaitEvent(pipe->out, computed, 0) != cudaSuccess ||
-          cudaMemcpyAsync(atw(h_o, qoff), at(d_o, qoff), qlen, cudaMemcpyDeviceToHost,
-                          pipe->out) != cudaSuccess)
-        return fail(BSATTN_ERR_CUDA);
+    for (int kv0 = 0; kv0 < Hkv; kv0 += hkc) {
+      const bool end = (b == 0 && kv0 == 0) || (b == B - 1 && kv0 + hkc == Hkv);
+      const int piece = split_ends && end ? 2 : hqc;   // query heads per piece
+      for (int h0 = 0; h0 < hqc; h0 += piece, ++c) {
+        const int hq0 = kv0 * G + h0;
+        const size_t qoff = ((size_t)b * Hq + hq0) * row, qlen = (size_t)piece * row;
+        const size_t koff = ((size_t)b * Hkv + kv0) * row, klen = (size_t)hkc * row;
+        cudaEvent_t copied = pipe->copied[c % kEvents], computed = pipe->computed[c % kEvents];
+        if (cudaMemcpyAsync(atw(d_q, qoff), at(h_q, qoff), qlen, cudaMemcpyHostToDevice,
+                            pipe->in) != cudaSuccess ||
+            (h0 == 0 && (cudaMemcpyAsync(atw(d_k, koff), at(h_k, koff), klen,
+                                         cudaMemcpyHostToDevice, pipe->in) != cudaSuccess ||
+                         cudaMemcpyAsync(atw(d_v, koff), at(h_v, koff), klen,
+                                         cudaMemcpyHostToDevice, pipe->in) != cudaSuccess)) ||
+            cudaEventRecord(copied, pipe->in) != cudaSuccess ||
+            cudaStreamWaitEvent(stream, copied, 0) != cudaSuccess)
+          return fail(BSATTN_ERR_CUDA);
+        // the piece as a problem of its own: one sequence, `piece` query
+        // heads of hkc KV heads; per-head CSR rows and orders start at its
+        // first head
+        const bool per_head = row_ptr && mask_heads == Hq;
+        const int rc = bsattn_fwd_prefill(
+            at(d_q, qoff), at(d_k, koff), at(d_v, koff), atw(d_o, qoff), nullptr, 1, piece, hkc, N,
+            d, block, scale, causal, lambda,
+            row_ptr ? row_ptr + (per_head ? (size_t)hq0 * (nq + 1) : 0) : nullptr, col_idx,
+            row_order ? row_order + (per_head ? (size_t)hq0 * nq : 0) : nullptr,
+            per_head ? piece : 1, nullptr, d_status, stream);
+        if (rc != BSATTN_OK) return fail(rc);
+        if (cudaEventRecord(computed, stream) != cudaSuccess ||
+            cudaStreamWaitEvent(pipe->out, computed, 0) != cudaSuccess ||
+            cudaMemcpyAsync(atw(h_o, qoff), at(d_o, qoff), qlen, cudaMemcpyDeviceToHost,
+                            pipe->out) != cudaSuccess)
+          return fail(BSATTN_ERR_CUDA);
+      }
     }
   }
   // the caller's stream completes after the last copy out

@@ -214,8 +214,12 @@ int bsattn_fwd_prefill_ex(const void *q, const void *k, const void *v, void *o, 
  * heads (with their query heads); each chunk is copied host -> device on an
  * internal stream, computed by bsattn_fwd_prefill on `stream` once its copies
  * have landed, and its O copied device -> host on a second internal stream,
- * so copies in, kernels and copies out of different chunks run at once.  The
- * call only enqueues work: `stream` completes after the last copy out.
+ * so copies in, kernels and copies out of different chunks run at once.  With
+ * one KV head per chunk and an even group of at least 4 query heads, the
+ * first and the last chunk run as pieces of 2 query heads (the first piece
+ * brings the KV head's K and V), which shortens the two ends the copies in
+ * cannot hide.  The call only enqueues work: `stream` completes after the
+ * last copy out.
  *
  *   h_q, h_k, h_v   host inputs, layouts as in bsattn_fwd_prefill; page-locked
  *                   (cudaHostAlloc / pinned) for the copies to overlap
