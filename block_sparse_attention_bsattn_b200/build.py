@@ -1,11 +1,16 @@
 """Build the CUDA library ``libbsattn.so`` for sm_100a with nvcc.
 
     python -m block_sparse_attention_bsattn_b200.build [--force] [--verbose]
+    python -m block_sparse_attention_bsattn_b200.build --probes
 
 Each ``csrc/*.cu`` is compiled to an object in ``_build/`` and the objects are
 linked into ``block_sparse_attention_bsattn_b200/lib/libbsattn.so`` (CUDA
 runtime linked statically, so the library does not depend on which libcudart
 the host process has loaded).  Rebuilds only what changed.
+
+``--probes`` builds the hardware microbenchmarks of ``probes/*.cu`` (MMA issue
+rate, TMEM read cost, L2 -> SM stream rate, exponential rates) into
+``_build/probes/``; they are measurement programs, not part of the library.
 """
 from __future__ import annotations
 
@@ -24,6 +29,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libbsattn.so")
+PROBES = os.path.join(PKG, "probes")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -77,10 +83,31 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     return LIB
 
 
+def build_probes(verbose: bool = False) -> list:
+    out_dir = os.path.join(BUILD, "probes")
+    os.makedirs(out_dir, exist_ok=True)
+    cc = nvcc()
+    outs = []
+    for src in sorted(glob.glob(os.path.join(PROBES, "*.cu"))):
+        exe = os.path.join(out_dir, os.path.basename(src)[:-3])
+        cmd = [cc, *ARCH, "-O3", "-std=c++17", "-I", CSRC, src, "-o", exe, "-lcuda"]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"nvcc failed:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
+        outs.append(exe)
+    return outs
+
+
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true")
+    ap.add_argument("--probes", action="store_true", help="build probes/*.cu instead of the library")
     a = ap.parse_args()
-    print(build(a.force, a.verbose, a.ptxas_info))
+    if a.probes:
+        print("\n".join(build_probes(a.verbose)))
+    else:
+        print(build(a.force, a.verbose, a.ptxas_info))

@@ -271,6 +271,12 @@ __global__ void __launch_bounds__(384, 1)
           if (SKIPV) continue;   // warp 10 loads V
           const int vs = t % C::VST;
           if (!mbar_wait(&bars->v_empty[vs], ((t / C::VST) & 1) ^ 1, abort, lim)) break;
+          // with the vote, a step that both slots skip hands its V slot back
+          // without waiting for the tile: the previous load into the slot
+          // must have landed before the slot is armed again
+          if (VOTE && t >= C::VST &&
+              !mbar_wait(&bars->v_full[vs], ((t / C::VST) & 1) ^ 1, abort, lim))
+            break;
           mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
           for (int hf = 0; hf < C::HALVES; ++hf)
             tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
@@ -283,6 +289,10 @@ __global__ void __launch_bounds__(384, 1)
           for (int t = (issued_v > C::VST ? issued_v - C::VST : 0); t < issued_v; ++t)
             mbar_wait_drain(&bars->v_full[t % C::VST], (t / C::VST) & 1, lim);
           if (!p.debug_stall) mbar_wait_drain(&bars->q_full, 0, lim);
+        } else if (VOTE && !SKIPV) {
+          // V tiles of skipped steps nobody waited for land before the CTA exits
+          for (int t = (issued_v > C::VST ? issued_v - C::VST : 0); t < issued_v; ++t)
+            mbar_wait_drain(&bars->v_full[t % C::VST], (t / C::VST) & 1, lim);
         }
       }
     } else if (SKIPV && warp == 2) {
@@ -402,13 +412,16 @@ __global__ void __launch_bounds__(384, 1)
           }
           if (!ok) break;
           if (more) mma_commit(&bars->k_empty[(t + 1) % C::KST]);
-          // release V_t: consumed (or not needed) by both heads; with V skipping
-          // a step that no slot keeps has no V tile
+          // release V_t: consumed (or not needed) by both slots; with V skipping
+          // a step that no slot keeps has no V tile.  With the vote, a step
+          // that no slot keeps releases the slot at once, without waiting for
+          // the tile to land (the producer waits for that before it loads the
+          // slot again), so the MMA warp goes straight on to the next step.
           if (v_ready) {
             mma_commit(&bars->v_empty[vs]);
             ++vc;
           } else if (!SKIPV) {
-            if (!mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) break;
+            if (!VOTE && !mbar_wait(&bars->v_full[vs], (t / C::VST) & 1, abort, lim)) break;
             mbar_arrive(&bars->v_empty[vs]);
           }
         }

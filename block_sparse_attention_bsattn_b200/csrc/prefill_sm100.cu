@@ -234,6 +234,11 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
         if (SKIPV) continue;   // warp 10 loads V
         const int vs = t % C::VST;
         if (!mbar_wait(&bars->v_empty[vs], ((t / C::VST) & 1) ^ 1, abort, lim)) break;
+        // a skipped tile hands its V slot back without waiting for the tile:
+        // the previous load into the slot must have landed before it is armed
+        if (p.use_skip && t >= C::VST &&
+            !mbar_wait(&bars->v_full[vs], ((t / C::VST) & 1) ^ 1, abort, lim))
+          break;
         mbar_arrive_expect_tx(&bars->v_full[vs], C::T_BYTES);
         for (int hf = 0; hf < C::HALVES; ++hf)
           tma_load_3d(v_smem + vs * C::T_BYTES + hf * C::T_HALF, &tmV, &bars->v_full[vs],
@@ -244,6 +249,10 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
         // let every copy this thread started land before the CTA can exit
         for (int t = (issued_k > C::KST ? issued_k - C::KST : 0); t < issued_k; ++t)
           mbar_wait_drain(&bars->k_full[t % C::KST], (t / C::KST) & 1, lim);
+        for (int t = (issued_v > C::VST ? issued_v - C::VST : 0); t < issued_v; ++t)
+          mbar_wait_drain(&bars->v_full[t % C::VST], (t / C::VST) & 1, lim);
+      } else if (p.use_skip && !SKIPV) {
+        // V tiles of skipped tiles nobody waited for land before the CTA exits
         for (int t = (issued_v > C::VST ? issued_v - C::VST : 0); t < issued_v; ++t)
           mbar_wait_drain(&bars->v_full[t % C::VST], (t / C::VST) & 1, lim);
       }
@@ -307,8 +316,8 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
         // V ring position: every visited tile's, or (V skipping) the kept ones'
         const int vi = SKIPV ? kept : t;
         const int vs = vi % C::VST;
-        if ((!SKIPV || !skip) && !mbar_wait(&bars->v_full[vs], (vi / C::VST) & 1, abort, lim))
-          break;
+        // a skipped tile does not wait for its V tile (see the producer)
+        if (!skip && !mbar_wait(&bars->v_full[vs], (vi / C::VST) & 1, abort, lim)) break;
         tc_fence_after();
         if (!skip) {
           const uint32_t p_tmem = tmem + C::S_COL + (uint32_t)sb * 128u;
