@@ -42,6 +42,7 @@
 
 #include "backward_internal.h"
 #include "sm100_ptx.cuh"
+#include "umma_desc.cuh"
 
 namespace bsattn {
 
@@ -276,25 +277,26 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t k_addr = smem_u32(smem + C::KV_K);
-      const uint32_t v_addr = smem_u32(smem + C::KV_V);
+      const uint64_t k_desc = smem_desc(smem_u32(smem + C::KV_K), 16, 1024, 2);
+      const uint64_t v_desc = smem_desc(smem_u32(smem + C::KV_V), 16, 1024, 2);
+      const uint64_t stg_desc = smem_desc(smem_u32(smem + C::KV_STG), 16, 1024, 2);
+      const uint64_t stg_desc_mn = smem_desc(smem_u32(smem + C::KV_STG), C::T_HALF, 1024, 2);
       // S^T and dP^T of half x (queries 64 (x & 1) .. + 64 of the pair in
       // stage st): keys on the rows, the half's queries on the columns
       auto first = [&](int x, int st) {
         const uint32_t buf = tmem + C::BUF + 128u * (uint32_t)(x & 1);
-        const uint32_t qa = smem_u32(smem + C::KV_STG + st * C::KV_STG_BYTES) + (x & 1) * 8192;
-        const uint32_t da = qa + C::T_BYTES;
+        const uint64_t qd = desc_add(stg_desc, st * C::KV_STG_BYTES + (x & 1) * 8192);
+        const uint64_t dd = desc_add(qd, C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(buf, smem_desc(k_addr + off, 16, 1024, 2), smem_desc(qa + off, 16, 1024, 2),
-                 IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(buf, desc_add(k_desc, off), desc_add(qd, off), IDESC_S, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(buf + C::DPOFF, smem_desc(v_addr + off, 16, 1024, 2),
-                 smem_desc(da + off, 16, 1024, 2), IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(buf + C::DPOFF, desc_add(v_desc, off), desc_add(dd, off), IDESC_S,
+                 kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars->s_full[x & 1]);
       };
@@ -305,18 +307,16 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(&bars->p_ready[x & 1], (x >> 1) & 1, abort, lim)) return false;
         tc_fence_after();
         const uint32_t buf = tmem + C::BUF + 128u * (uint32_t)(x & 1);
-        const uint32_t qa = smem_u32(smem + C::KV_STG + st * C::KV_STG_BYTES) + (x & 1) * 8192;
-        const uint32_t da = qa + C::T_BYTES;
+        const uint64_t qd = desc_add(stg_desc_mn, st * C::KV_STG_BYTES + (x & 1) * 8192);
+        const uint64_t dd = desc_add(qd, C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 64 / 16; ++kk)
-          mma_ts(tmem + C::ACC1, buf + bf16_col(kk),
-                 smem_desc(da + kk * (16 * 128), C::T_HALF, 1024, 2), IDESC_O,
+          mma_ts(tmem + C::ACC1, buf + bf16_col(kk), desc_add(dd, kk * (16 * 128)), IDESC_O,
                  (x > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 64 / 16; ++kk)
-          mma_ts(tmem + C::ACC0, buf + C::DPOFF + bf16_col(kk),
-                 smem_desc(qa + kk * (16 * 128), C::T_HALF, 1024, 2), IDESC_O,
-                 (x > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + C::ACC0, buf + C::DPOFF + bf16_col(kk), desc_add(qd, kk * (16 * 128)),
+                 IDESC_O, (x > 0 || kk > 0) ? 1u : 0u);
         if (x & 1) mma_commit(&bars->st_empty[st]);
         return true;
       };
@@ -582,24 +582,25 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_addr = smem_u32(smem + C::Q_Q);
-      const uint32_t do_addr = smem_u32(smem + C::Q_DO);
+      const uint64_t q_desc = smem_desc(smem_u32(smem + C::Q_Q), 16, 1024, 2);
+      const uint64_t do_desc = smem_desc(smem_u32(smem + C::Q_DO), 16, 1024, 2);
+      const uint64_t stg_desc = smem_desc(smem_u32(smem + C::Q_STG), 16, 1024, 2);
+      const uint64_t stg_desc_mn = smem_desc(smem_u32(smem + C::Q_STG), C::T_HALF, 1024, 2);
       // S and dP of half x (keys 64 (x & 1) .. + 64 of the key tile in stage st)
       auto first = [&](int x, int st) {
         const uint32_t buf = tmem + C::BUF + 128u * (uint32_t)(x & 1);
-        const uint32_t ka = smem_u32(smem + C::Q_STG + st * C::Q_STG_BYTES) + (x & 1) * 8192;
-        const uint32_t va = ka + C::T_BYTES;
+        const uint64_t kd = desc_add(stg_desc, st * C::Q_STG_BYTES + (x & 1) * 8192);
+        const uint64_t vd = desc_add(kd, C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(buf, smem_desc(q_addr + off, 16, 1024, 2), smem_desc(ka + off, 16, 1024, 2),
-                 IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(buf, desc_add(q_desc, off), desc_add(kd, off), IDESC_S, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(buf + C::DPOFF, smem_desc(do_addr + off, 16, 1024, 2),
-                 smem_desc(va + off, 16, 1024, 2), IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(buf + C::DPOFF, desc_add(do_desc, off), desc_add(vd, off), IDESC_S,
+                 kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars->s_full[x & 1]);
       };
@@ -610,11 +611,10 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(&bars->p_ready[x & 1], (x >> 1) & 1, abort, lim)) return false;
         tc_fence_after();
         const uint32_t buf = tmem + C::BUF + 128u * (uint32_t)(x & 1);
-        const uint32_t ka = smem_u32(smem + C::Q_STG + st * C::Q_STG_BYTES) + (x & 1) * 8192;
+        const uint64_t kd = desc_add(stg_desc_mn, st * C::Q_STG_BYTES + (x & 1) * 8192);
 #pragma unroll
         for (int kk = 0; kk < 64 / 16; ++kk)
-          mma_ts(tmem + C::ACC0, buf + bf16_col(kk),
-                 smem_desc(ka + kk * (16 * 128), C::T_HALF, 1024, 2), IDESC_O,
+          mma_ts(tmem + C::ACC0, buf + bf16_col(kk), desc_add(kd, kk * (16 * 128)), IDESC_O,
                  (x > 0 || kk > 0) ? 1u : 0u);
         if (x & 1) mma_commit(&bars->st_empty[st]);
         return true;

@@ -43,6 +43,7 @@
 
 #include "bsattn_internal.h"
 #include "sm100_ptx.cuh"
+#include "umma_desc.cuh"
 
 namespace bsattn {
 
@@ -286,8 +287,8 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
     if (lane == 0 && n > 0) {
       constexpr uint32_t IDESC1 = idesc_bf16_f32(128, BLK, 0, 0);
       constexpr uint32_t IDESC2 = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t k_addr = smem_u32(k_smem);
-      const uint32_t v_addr = smem_u32(v_smem);
+      const uint64_t k_desc = smem_desc(smem_u32(k_smem), 16, 1024, 2);
+      const uint64_t v_desc = smem_desc(smem_u32(v_smem), C::T_HALF, 1024, 2);
       bool ok = mbar_wait(&bars->q_ready, 0, abort, lim);
       tc_fence_after();
       auto issue_bmm1 = [&](int t) -> bool {
@@ -295,12 +296,11 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
         if (!mbar_wait(&bars->k_full[ks], (t / C::KST) & 1, abort, lim)) return false;
         tc_fence_after();
         const uint32_t d_tmem = tmem + C::S_COL + (uint32_t)(t & 1) * 128u;
+        const uint64_t kd = desc_add(k_desc, ks * C::T_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t bb = k_addr + ks * C::T_BYTES + (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ts(d_tmem, tmem + C::Q_COL + kk * 8, smem_desc(bb, 16, 1024, 2), IDESC1,
-                 kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ts(d_tmem, tmem + C::Q_COL + kk * 8, desc_add(kd, (kk / 4) * C::T_HALF + (kk % 4) * 32),
+                 IDESC1, kk > 0 ? 1u : 0u);
         mma_commit(&bars->s_full[t & 1]);
         mma_commit(&bars->k_empty[ks]);
         return true;
@@ -321,12 +321,11 @@ __global__ void __launch_bounds__(SKIPV ? 352 : 320, 1)
         tc_fence_after();
         if (!skip) {
           const uint32_t p_tmem = tmem + C::S_COL + (uint32_t)sb * 128u;
+          const uint64_t vd = desc_add(v_desc, vs * C::T_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BLK / 16; ++kk) {
-            const uint32_t bb = v_addr + vs * C::T_BYTES + kk * (16 * 128);
-            mma_ts(tmem + C::O_COL, p_tmem + kk * 8, smem_desc(bb, C::T_HALF, 1024, 2), IDESC2,
+          for (int kk = 0; kk < BLK / 16; ++kk)
+            mma_ts(tmem + C::O_COL, p_tmem + kk * 8, desc_add(vd, kk * (16 * 128)), IDESC2,
                    (kept > 0 || kk > 0) ? 1u : 0u);
-          }
           mma_commit(&bars->o_done);
           mma_commit(&bars->v_empty[vs]);
           ++kept;
