@@ -106,6 +106,37 @@ def test_blasst_random_masks_per_head(d, block):
     assert torch.isneginf(lse[:, :, rows]).all()
 
 
+@pytest.mark.parametrize("d,block", [(64, 64), (128, 128)])
+@pytest.mark.parametrize("lam", [0.0, 3e-3])
+def test_running_max_jumps_in_a_later_tile(d, block, lam):
+    """Scores that jump far beyond the lazy-rescale slack (8 in base 2) in a
+    later key tile: in the low half of key tile 2's columns for the first half
+    of the last query tile's rows, in the high half of key tile 3 for the
+    rest.  The exponent shift then moves after the first kept tile, so the
+    one-tile kernel's exponentials taken before the two column halves have
+    exchanged their maxima must be redone for those rows (one query head per
+    KV head, per-head all-ones masks: the one-tile kernel)."""
+    B, Hq, Hkv, nt = 1, 2, 2, 5
+    N = nt * block
+    q, k, v = inputs.normal_qkv(B, Hq, Hkv, N, d, "cpu", 321 + d)
+    scale = 1 / math.sqrt(d)
+    qf, kf = q.float(), k.float()
+    r0 = (nt - 1) * block
+    for h in range(Hq):
+        for r in range(block):
+            key = (2 * block + r) if r < block // 2 else (3 * block + r)
+            qr = qf[0, h, r0 + r]
+            kf[0, h, key] = qr * (20.0 / (scale * float(qr @ qr)))   # score 20 for this row
+    k = kf.to(torch.bfloat16)
+    w = inputs.Workload("jump", B, Hq, Hkv, N, d, block, False, "prefill", scale, None,
+                        q=q, k=k, v=v)
+    nb = nt
+    mask = np.ones((Hq, nb, nb), dtype=np.uint8)
+    ref = _check(w, lam, mask, f"jump d{d} b{block} lam{lam}")
+    # the jump really happened: the last tile's rows end far above their first tile's max
+    assert (ref["lse"][0, :, r0:] > 15).all()
+
+
 @pytest.mark.parametrize("a", [0.0, 10.0, 1000.0])
 def test_blasst_prefill_one_head_per_kv_head(a):
     """Causal BLASST prefill with one query head per KV head and several
