@@ -101,6 +101,21 @@ struct PairBarriers {
   int dval[2][4];           // 1 = kept
 };
 
+// A shared-memory matrix descriptor (the layout of smem_desc) as its two
+// 32-bit words: the low word holds the start address and the leading offset,
+// the high word only constants (stride offset, version, swizzle), so the
+// descriptor of a tile `off` bytes further on is the low word plus off / 16
+// (addresses stay below 256 KB: no carry out of the 14-bit address field).
+__host__ __device__ constexpr uint32_t desc_hi(uint32_t sbo_bytes, uint32_t swizzle) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | ((swizzle & 0x7u) << 29);
+}
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t desc_of(uint32_t lo, uint32_t hi) {
+  return ((uint64_t)hi << 32) | lo;
+}
+
 template <int D, bool SKIPV, bool VOTE>
 __global__ void __launch_bounds__(384, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -333,31 +348,32 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0 && n > 0) {
         constexpr uint32_t IDESC1 = idesc_bf16_f32(128, BLK, 0, 0);
         constexpr uint32_t IDESC2 = idesc_bf16_f32(128, D, 0, 1);
-        const uint32_t q_addr = smem_u32(q_smem);
-        const uint32_t k_addr = smem_u32(k_smem);
-        const uint32_t v_addr = smem_u32(v_smem);
+        constexpr uint32_t HI = desc_hi(1024, 2);
+        const uint32_t q_lo = desc_lo(smem_u32(q_smem), 16);
+        const uint32_t k_lo = desc_lo(smem_u32(k_smem), 16);
+        const uint32_t v_lo = desc_lo(smem_u32(v_smem), C::T_HALF);
         bool ok = mbar_wait(&bars->q_full, 0, abort, lim);
         tc_fence_after();
         // S_e = Q_e K_t^T into TMEM columns [256 e, 256 e + 128)
         auto bmm1 = [&](int e, int t) {
-          const int ks = t % C::KST;
+          const uint32_t qa = q_lo + (uint32_t)e * (C::Q_BYTES / 16);
+          const uint32_t ka = k_lo + (uint32_t)(t % C::KST) * (C::T_BYTES / 16);
   #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t a = q_addr + e * C::Q_BYTES + (kk / 4) * C::Q_HALF + (kk % 4) * 32;
-            const uint32_t bb = k_addr + ks * C::T_BYTES + (kk / 4) * C::T_HALF + (kk % 4) * 32;
-            mma_ss(tmem + 256 * e, smem_desc(a, 16, 1024, 2), smem_desc(bb, 16, 1024, 2), IDESC1,
+            const uint32_t qo = ((kk / 4) * C::Q_HALF + (kk % 4) * 32) / 16;
+            const uint32_t ko = ((kk / 4) * C::T_HALF + (kk % 4) * 32) / 16;
+            mma_ss(tmem + 256 * e, desc_of(qa + qo, HI), desc_of(ka + ko, HI), IDESC1,
                    kk > 0 ? 1u : 0u);
           }
           mma_commit(&bars->s_full[e]);
         };
         // O_e += P_e V, P_e in TMEM over S_e, V in ring slot vs
         auto bmm2 = [&](int e, int vs, int first) {
+          const uint32_t va = v_lo + (uint32_t)vs * (C::T_BYTES / 16);
   #pragma unroll
-          for (int kk = 0; kk < BLK / 16; ++kk) {
-            const uint32_t bb = v_addr + vs * C::T_BYTES + kk * (16 * 128);
-            mma_ts(tmem + 256 * e + 128, tmem + 256 * e + kk * 8, smem_desc(bb, C::T_HALF, 1024, 2),
+          for (int kk = 0; kk < BLK / 16; ++kk)
+            mma_ts(tmem + 256 * e + 128, tmem + 256 * e + kk * 8, desc_of(va + kk * (16 * 128) / 16, HI),
                    IDESC2, (!first || kk > 0) ? 1u : 0u);
-          }
           mma_commit(&bars->o_done[e]);
         };
         if (ok) {
