@@ -277,25 +277,25 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
-      const uint64_t k_desc = smem_desc(smem_u32(smem + C::KV_K), 16, 1024, 2);
-      const uint64_t v_desc = smem_desc(smem_u32(smem + C::KV_V), 16, 1024, 2);
-      const uint64_t stg_desc = smem_desc(smem_u32(smem + C::KV_STG), 16, 1024, 2);
-      const uint64_t stg_desc_mn = smem_desc(smem_u32(smem + C::KV_STG), C::T_HALF, 1024, 2);
+      const uint32_t k_lo = udesc_lo(smem_u32(smem + C::KV_K), 16);
+      const uint32_t v_lo = udesc_lo(smem_u32(smem + C::KV_V), 16);
+      const uint32_t stg_lo = udesc_lo(smem_u32(smem + C::KV_STG), 16);
+      const uint32_t stg_lo_mn = udesc_lo(smem_u32(smem + C::KV_STG), C::T_HALF);
       // S^T and dP^T of half x (queries 64 (x & 1) .. + 64 of the pair in
       // stage st): keys on the rows, the half's queries on the columns
       auto first = [&](int x, int st) {
         const uint32_t buf = tmem + C::BUF + 128u * (uint32_t)(x & 1);
-        const uint64_t qd = desc_add(stg_desc, st * C::KV_STG_BYTES + (x & 1) * 8192);
-        const uint64_t dd = desc_add(qd, C::T_BYTES);
+        const uint32_t qd = udesc_step(stg_lo, st * C::KV_STG_BYTES + (x & 1) * 8192);
+        const uint32_t dd = udesc_step(qd, C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(buf, desc_add(k_desc, off), desc_add(qd, off), IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(buf, udesc128(k_lo, off), udesc128(qd, off), IDESC_S, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(buf + C::DPOFF, desc_add(v_desc, off), desc_add(dd, off), IDESC_S,
+          mma_ss(buf + C::DPOFF, udesc128(v_lo, off), udesc128(dd, off), IDESC_S,
                  kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars->s_full[x & 1]);
@@ -307,15 +307,15 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(&bars->p_ready[x & 1], (x >> 1) & 1, abort, lim)) return false;
         tc_fence_after();
         const uint32_t buf = tmem + C::BUF + 128u * (uint32_t)(x & 1);
-        const uint64_t qd = desc_add(stg_desc_mn, st * C::KV_STG_BYTES + (x & 1) * 8192);
-        const uint64_t dd = desc_add(qd, C::T_BYTES);
+        const uint32_t qd = udesc_step(stg_lo_mn, st * C::KV_STG_BYTES + (x & 1) * 8192);
+        const uint32_t dd = udesc_step(qd, C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 64 / 16; ++kk)
-          mma_ts(tmem + C::ACC1, buf + bf16_col(kk), desc_add(dd, kk * (16 * 128)), IDESC_O,
+          mma_ts(tmem + C::ACC1, buf + bf16_col(kk), udesc128(dd, kk * (16 * 128)), IDESC_O,
                  (x > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 64 / 16; ++kk)
-          mma_ts(tmem + C::ACC0, buf + C::DPOFF + bf16_col(kk), desc_add(qd, kk * (16 * 128)),
+          mma_ts(tmem + C::ACC0, buf + C::DPOFF + bf16_col(kk), udesc128(qd, kk * (16 * 128)),
                  IDESC_O, (x > 0 || kk > 0) ? 1u : 0u);
         if (x & 1) mma_commit(&bars->st_empty[st]);
         return true;
@@ -582,24 +582,24 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);
-      const uint64_t q_desc = smem_desc(smem_u32(smem + C::Q_Q), 16, 1024, 2);
-      const uint64_t do_desc = smem_desc(smem_u32(smem + C::Q_DO), 16, 1024, 2);
-      const uint64_t stg_desc = smem_desc(smem_u32(smem + C::Q_STG), 16, 1024, 2);
-      const uint64_t stg_desc_mn = smem_desc(smem_u32(smem + C::Q_STG), C::T_HALF, 1024, 2);
+      const uint32_t q_lo = udesc_lo(smem_u32(smem + C::Q_Q), 16);
+      const uint32_t do_lo = udesc_lo(smem_u32(smem + C::Q_DO), 16);
+      const uint32_t stg_lo = udesc_lo(smem_u32(smem + C::Q_STG), 16);
+      const uint32_t stg_lo_mn = udesc_lo(smem_u32(smem + C::Q_STG), C::T_HALF);
       // S and dP of half x (keys 64 (x & 1) .. + 64 of the key tile in stage st)
       auto first = [&](int x, int st) {
         const uint32_t buf = tmem + C::BUF + 128u * (uint32_t)(x & 1);
-        const uint64_t kd = desc_add(stg_desc, st * C::Q_STG_BYTES + (x & 1) * 8192);
-        const uint64_t vd = desc_add(kd, C::T_BYTES);
+        const uint32_t kd = udesc_step(stg_lo, st * C::Q_STG_BYTES + (x & 1) * 8192);
+        const uint32_t vd = udesc_step(kd, C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(buf, desc_add(q_desc, off), desc_add(kd, off), IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(buf, udesc128(q_lo, off), udesc128(kd, off), IDESC_S, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::T_HALF + (kk % 4) * 32;
-          mma_ss(buf + C::DPOFF, desc_add(do_desc, off), desc_add(vd, off), IDESC_S,
+          mma_ss(buf + C::DPOFF, udesc128(do_lo, off), udesc128(vd, off), IDESC_S,
                  kk > 0 ? 1u : 0u);
         }
         mma_commit(&bars->s_full[x & 1]);
@@ -611,10 +611,10 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(&bars->p_ready[x & 1], (x >> 1) & 1, abort, lim)) return false;
         tc_fence_after();
         const uint32_t buf = tmem + C::BUF + 128u * (uint32_t)(x & 1);
-        const uint64_t kd = desc_add(stg_desc_mn, st * C::Q_STG_BYTES + (x & 1) * 8192);
+        const uint32_t kd = udesc_step(stg_lo_mn, st * C::Q_STG_BYTES + (x & 1) * 8192);
 #pragma unroll
         for (int kk = 0; kk < 64 / 16; ++kk)
-          mma_ts(tmem + C::ACC0, buf + bf16_col(kk), desc_add(kd, kk * (16 * 128)), IDESC_O,
+          mma_ts(tmem + C::ACC0, buf + bf16_col(kk), udesc128(kd, kk * (16 * 128)), IDESC_O,
                  (x > 0 || kk > 0) ? 1u : 0u);
         if (x & 1) mma_commit(&bars->st_empty[st]);
         return true;
